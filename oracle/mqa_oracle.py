@@ -1,0 +1,165 @@
+"""CPU float64 oracle for single-token incremental-decode attention over a KV cache.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports this module; only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+call it.  It shares no code with the CUDA path: it reads plain NumPy arrays and
+writes plain NumPy arrays, and it is written straight from the definitions on
+the pages, without blocking, splitting or reordering.
+
+Sources (web pages on Multi-Query Attention; cited by title and section):
+
+* [velog review] "[Paper review] Fast Transformer Decoding: One Write-Head is All
+  You Need", §2.1 (DotProductAttention), §2.4 (MultiheadSelfAttentionIncremental)
+  and §3 (MultiquerySelfAttentionIncremental).  These give the computation as
+  einsums: logits = einsum("bhk,bmk->bhm", q, K); weights = softmax(logits);
+  o = einsum("bhm,bmv->bhv", weights, V); the per-head form has K/V [b,h,m,k].
+* [kuangjux notes] "Fast Transformer Decoding: One Write-Head is All You Need"
+  (study notes), §1 (the scaled, masked softmax O = softmax(QKᵀ/√d_h + M)V) and
+  §4 (MQA drops only the head axis of K/V; worked example with two keys).
+* [oscine blog] "GQA、MQA、MLA：当「多头」变成推理账单上最贵的一项", section
+  "第三站: GQA" (H query heads split into G groups, one K/V head per group;
+  GQA-1 is MQA, GQA-H is MHA).
+
+Readings where the pages leave a step open (each listed again in the design
+notes of the repository):
+
+* Scale: the pseudocode has none, the notes divide by √d_h.  Every function here
+  takes ``scale`` and multiplies the logits by it; callers pick the value.
+* Mask: position t of sequence b is valid iff t < lens[b] (the query is the
+  newest token, so causality is implied).  Rows at t >= lens[b] are never read,
+  so their contents (NaN in the tests) cannot leak into the result.
+* Grouping: query head i reads K/V head j(i) = i // (h // g), i.e. contiguous
+  groups; h must be a multiple of g.
+* lens[b] == 0: the output row is 0 and lse is -inf (the pages do not define it).
+
+Parity pins for every function live in ``tests/test_oracle.py``; none is
+unpinned.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "dot_product_attention",
+    "oracle_decode",
+    "oracle_kv_append",
+    "oracle_decode_step",
+]
+
+
+def dot_product_attention(q, K, V, scale=1.0):
+    """Attention for ONE query against one K/V head, with plain Python loops.
+
+    Follows [velog review] §2.1 DotProductAttention: q [k], K [m, k], V [m, v];
+    logits_t = Σ_r q_r K_{t,r}; weights = softmax(logits); y = Σ_t w_t V_t.
+    The scale multiplies the logits (the √d_h division of [kuangjux notes] §1).
+    Small inputs only: this is the brute-force reference the batched oracle is
+    checked against.
+    """
+    q = [float(x) for x in np.asarray(q, dtype=np.float64).ravel()]
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    m = K.shape[0]
+    logits = []
+    for t in range(m):
+        acc = 0.0
+        for r in range(len(q)):
+            acc += q[r] * float(K[t, r])
+        logits.append(acc * scale)
+    top = max(logits)
+    exps = [math.exp(s - top) for s in logits]
+    total = math.fsum(exps)
+    weights = [e / total for e in exps]
+    y = []
+    for c in range(V.shape[1]):
+        y.append(math.fsum(weights[t] * float(V[t, c]) for t in range(m)))
+    return np.array(y, dtype=np.float64), np.array(weights, dtype=np.float64)
+
+
+def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
+    """One decode step of MQA / GQA / MHA attention, in float64.
+
+    Shapes: q [b, h, d_k]; k_cache [b, m_max, g, d_k]; v_cache [b, m_max, g, d_v];
+    lens int [b].  Returns o [b, h, d_v] float64 and lse [b, h] float64 (natural
+    log of Σ_t exp(logit_t)), plus the weights as a list of [h, lens[b]] arrays
+    when ``return_weights``.
+
+    For each sequence b and K/V group j, the h//g query heads of that group form
+    a matrix Q_j [h//g, d_k]; with L = lens[b] and K_j = k_cache[b, :L, j, :]:
+        S = scale · Q_j K_jᵀ                       ([velog review] §3 logits einsum)
+        w = softmax over the L valid positions      (§3 softmax; [kuangjux notes] §1)
+        o = w V_j                                   (§3 weighted-V einsum)
+    g = 1 is MQA, g = h is MHA, 1 < g < h is GQA ([oscine blog] "第三站: GQA").
+    Inputs are used at whatever precision they hold (the tests hand in values
+    already rounded to the kernel's input type) and widened to float64 here.
+    """
+    q = np.asarray(q)
+    k_cache = np.asarray(k_cache)
+    v_cache = np.asarray(v_cache)
+    lens = np.asarray(lens).astype(np.int64)
+    b, h, d_k = q.shape
+    _, m_max, g_cache, _ = k_cache.shape
+    d_v = v_cache.shape[3]
+    if g_cache != g or h % g != 0:
+        raise ValueError("k_cache must have g heads and h must be a multiple of g")
+    hq = h // g
+    o = np.zeros((b, h, d_v), dtype=np.float64)
+    lse = np.full((b, h), -np.inf, dtype=np.float64)
+    weights = [] if return_weights else None
+    for bi in range(b):
+        L = int(lens[bi])
+        if L > m_max:
+            raise ValueError("lens[b] exceeds m_max")
+        w_b = np.zeros((h, max(L, 0)), dtype=np.float64)
+        if L <= 0:
+            if return_weights:
+                weights.append(w_b)
+            continue
+        for j in range(g):
+            Qj = q[bi, j * hq:(j + 1) * hq, :].astype(np.float64)          # [hq, d_k]
+            Kj = k_cache[bi, :L, j, :].astype(np.float64)                   # [L, d_k]
+            Vj = v_cache[bi, :L, j, :].astype(np.float64)                   # [L, d_v]
+            S = scale * (Qj @ Kj.T)                                         # [hq, L]
+            mu = S.max(axis=1, keepdims=True)
+            E = np.exp(S - mu)
+            denom = E.sum(axis=1, keepdims=True)
+            W = E / denom
+            o[bi, j * hq:(j + 1) * hq, :] = W @ Vj
+            lse[bi, j * hq:(j + 1) * hq] = (mu + np.log(denom))[:, 0]
+            w_b[j * hq:(j + 1) * hq, :] = W
+        if return_weights:
+            weights.append(w_b)
+    if return_weights:
+        return o, lse, weights
+    return o, lse
+
+
+def oracle_kv_append(k_cache, v_cache, k_new, v_new, pos):
+    """The step's K/V written into the cache: the "one write-head".
+
+    [velog review] §3 builds new_K = concat([prev_K, k_new], axis=1) (and the same
+    for V).  With a fixed-size cache [b, m_max, g, d] the concat becomes a write
+    of k_new[b] at row pos[b] of sequence b; every other element is unchanged.
+    Returns new arrays (the inputs are not modified).  Works on any dtype,
+    including the raw bf16 bit patterns (uint16), so the comparison is bitwise.
+    """
+    k_out = np.array(k_cache, copy=True)
+    v_out = np.array(v_cache, copy=True)
+    pos = np.asarray(pos).astype(np.int64)
+    for bi in range(k_out.shape[0]):
+        p = int(pos[bi])
+        if 0 <= p < k_out.shape[1]:
+            k_out[bi, p] = k_new[bi]
+            v_out[bi, p] = v_new[bi]
+    return k_out, v_out
+
+
+def oracle_decode_step(q, k_cache, v_cache, k_new, v_new, lens_before, g, scale):
+    """One whole incremental step in the order of [velog review] §3: append the
+    new K/V at row lens_before[b], then attend over lens_before[b] + 1 rows."""
+    k2, v2 = oracle_kv_append(k_cache, v_cache, k_new, v_new, lens_before)
+    lens_after = np.asarray(lens_before).astype(np.int64) + 1
+    o, lse = oracle_decode(q, k2, v2, lens_after, g, scale)
+    return o, lse, k2, v2
