@@ -1,0 +1,408 @@
+"""Decode-attention benchmark: query-tokens/s and achieved HBM bandwidth of one
+decode step (append the step's K/V, then attend over every valid row) on the
+long-context MQA serving batch (b=64 sequences, h=32 query heads sharing one
+K/V head, d=128, m_max=8192, lengths uniform in [1024, 8192]).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  Under torchrun each rank runs the same
+per-GPU workload on its own GPU (weak scaling: sequences are independent, so
+no collective sits on the data path); the timed region is bracketed by a
+barrier and a device synchronize, and the step time is the maximum over ranks.
+``--impl reference`` times the CPU float64 oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from grouped_query_attention_mqa_b200.workloads import (WORKLOADS, append_algorithmic_bytes,  # noqa: E402
+                                                         decode_algorithmic_bytes, draw_lens, f32_to_bf16_bits,
+                                                         bf16_bits_to_f32)
+
+METRIC = "decode-attention achieved HBM GB/s vs peak; query-tokens/s at MQA b=64 m=8K"
+UNIT = "query-tokens/s"
+DEFAULT_WORKLOAD = "long_mqa_b64_m8k"
+SEED = 3
+L2_BYTES = 126 * 2**20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=200)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
+    p.add_argument("--num-ctas", type=int, default=0)
+    p.add_argument("--e2e-steps", type=int, default=2000)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ CPU side
+
+def cpu_sample(wl, seed, n_seq):
+    """A bounded sample of the workload for the oracle: the first n_seq
+    sequences with the workload's lengths, each holding only its valid rows
+    (bf16-rounded N(0,1) values, like the device inputs)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens = draw_lens(wl, rng)[:n_seq]
+    seqs = []
+    for L in lens:
+        def draw(shape, std=1.0):
+            x = rng.standard_normal(shape, dtype=np.float32) * np.float32(std)
+            return bf16_bits_to_f32(f32_to_bf16_bits(x)) if wl.dtype == "bf16" else x
+        seqs.append(dict(L=int(L), k=draw((1, int(L) - 1, wl.g, wl.d_k)), v=draw((1, int(L) - 1, wl.g, wl.d_v)),
+                         q=draw((1, wl.h, wl.d_k), wl.q_std), k_new=draw((1, wl.g, wl.d_k)),
+                         v_new=draw((1, wl.g, wl.d_v))))
+    return seqs
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [x.get("num_threads", 0) for x in threadpool_info() if x.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(wl, seconds, n_seq=16):
+    """Oracle steps (append, then attend) over sampled sequences until about
+    `seconds` of CPU time has passed.  Returns (tokens/s, sequences, seconds)."""
+    from oracle import oracle_decode_step   # test infrastructure: only this leg of the bench runs it
+
+    seqs = cpu_sample(wl, SEED, n_seq)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for s in seqs:
+            # the cache holds L-1 rows; the step appends row L-1 and attends over L rows
+            cache_k = np.concatenate([s["k"], np.zeros((1, 1, wl.g, wl.d_k), np.float32)], axis=1)
+            cache_v = np.concatenate([s["v"], np.zeros((1, 1, wl.g, wl.d_v), np.float32)], axis=1)
+            oracle_decode_step(s["q"], cache_k, cache_v, s["k_new"], s["v_new"], np.array([s["L"] - 1]), wl.g,
+                               wl.scale)
+            done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done / el, done, el
+
+
+def cpu_baseline_obj(wl, seconds):
+    v, n, el = time_oracle(wl, seconds)
+    return {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} sequence-steps of {wl.name} (first 16 sequences of seed {SEED}, valid rows only), "
+                      f"NumPy float64 append+attend, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        time_oracle(wl, 0.0, n_seq=2)
+    rates, total_n, total_t = [], 0, 0.0
+    for _ in range(args.steps):
+        v, n, el = time_oracle(wl, per_step)
+        rates.append(v)
+        total_n += n
+        total_t += el
+    value = total_n / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "b": wl.b, "h": wl.h, "g": wl.g, "d": wl.d_k, "m_max": wl.m_max,
+                       "lens": f"U[{wl.len_lo},{wl.len_hi}]", "step": "kv_append + decode"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{total_n} sequence-steps of {wl.name}, {per_step:.1f} s per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU side
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[3], 16)
+            except ValueError:
+                continue
+            for bit, name in self.REASONS.items():
+                if bits & bit:
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_digest(path_name):
+    files = ["common.cuh", "decode_tc.cu" if path_name == "tcgen05" else "decode_simt.cu", "merge.cu"]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "grouped_query_attention_mqa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, digest):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it stands (profiles/dram_traffic.txt)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload:
+            kv = dict(p.split("=", 1) for p in parts[2:] if "=" in p)
+            if kv.get("src_sha256") == digest:
+                return int(kv["bytes_per_launch"])
+    return None
+
+
+def resolve_path(binding, torch, requested):
+    if requested != "auto":
+        return requested
+    q = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 1, 128), dtype=torch.bfloat16, device="cuda")
+    try:
+        binding.decode(q, k, k, torch.ones(1, dtype=torch.int32, device="cuda"), 1.0, path="tcgen05")
+        return "tcgen05"
+    except binding.MqaError:
+        return "simt"
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from grouped_query_attention_mqa_b200 import binding
+    from grouped_query_attention_mqa_b200.build import LIB, build
+    from grouped_query_attention_mqa_b200.workloads import device_inputs
+
+    if not os.path.exists(LIB):
+        build()
+    binding.load_library()
+    wl = WORKLOADS[args.workload]
+    b, h, g, d = wl.b, wl.h, wl.g, wl.d_k
+    path = resolve_path(binding, torch, args.path)
+    cache_bytes = wl.b * wl.m_max * wl.g * (wl.d_k + wl.d_v) * wl.elem_bytes
+    copies = max(1, min(8, -(-3 * L2_BYTES // cache_bytes)))      # >= 3x L2 between reuses of one copy
+    inp = device_inputs(wl, seed=SEED + rank, device="cuda", copies=copies)
+    lens_np = inp["lens"]
+    lens = torch.from_numpy(lens_np).cuda()
+    pos = torch.from_numpy(lens_np - 1).cuda()
+    out = torch.empty((b, h, wl.d_v), dtype=inp["q"].dtype, device="cuda")
+    ws = torch.empty(binding.decode_workspace_size(b, h, g, wl.d_v), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    # one pre-marshalled append and decode per cache copy: each step is two C calls
+    appends = [binding.AppendPlan(inp["k"][c], inp["v"][c], inp["k_new"], inp["v_new"], pos) for c in range(copies)]
+    decodes = [binding.DecodePlan(inp["q"], inp["k"][c], inp["v"][c], lens, wl.scale, out=out, workspace=ws,
+                                  path=path, num_ctas=args.num_ctas) for c in range(copies)]
+
+    def step(i):
+        appends[i % copies].run()
+        decodes[i % copies].run()
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+
+    # timed region: K steps, events on the launching stream around the whole
+    # run and around every decode call
+    K = args.steps
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    time.sleep(0.2)
+    start.record(stream)
+    for i in range(K):
+        appends[i % copies].run()
+        ev_dec[i][0].record(stream)
+        decodes[i % copies].run()
+        ev_dec[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    dec_ms = [a.elapsed_time(z) for a, z in ev_dec]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    if world > 1:
+        t = torch.tensor([elapsed_ms, dec_avg_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_avg_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / K
+    value = world * b * K / (elapsed_ms / 1e3)
+
+    # end to end through the public API: pinned host inputs copied in, the
+    # step's output copied out, every step
+    E = args.e2e_steps
+    q_h = inp["q"].cpu().pin_memory()
+    kn_h = inp["k_new"].cpu().pin_memory()
+    vn_h = inp["v_new"].cpu().pin_memory()
+    lens_h = torch.from_numpy(lens_np).pin_memory()
+    pos_h = torch.from_numpy(lens_np - 1).pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, kn_d, vn_d = torch.empty_like(inp["q"]), torch.empty_like(inp["k_new"]), torch.empty_like(inp["v_new"])
+    lens_d, pos_d = torch.empty_like(lens), torch.empty_like(pos)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, kn_h, vn_h, lens_h, pos_h))
+    d2h = o_h.numel() * o_h.element_size()
+
+    e_app = [binding.AppendPlan(inp["k"][c], inp["v"][c], kn_d, vn_d, pos_d) for c in range(copies)]
+    e_dec = [binding.DecodePlan(q_d, inp["k"][c], inp["v"][c], lens_d, wl.scale, out=out, workspace=ws, path=path,
+                                num_ctas=args.num_ctas) for c in range(copies)]
+
+    def e2e_step(i):
+        q_d.copy_(q_h, non_blocking=True)
+        kn_d.copy_(kn_h, non_blocking=True)
+        vn_d.copy_(vn_h, non_blocking=True)
+        lens_d.copy_(lens_h, non_blocking=True)
+        pos_d.copy_(pos_h, non_blocking=True)
+        e_app[i % copies].run()
+        e_dec[i % copies].run()
+        o_h.copy_(out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for i in range(E):
+        e2e_step(i)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * b * E / (e2e_ms / 1e3)
+
+    alg_bytes = decode_algorithmic_bytes(wl, lens_np)
+    peak, peak_kind = peaks()
+    achieved = alg_bytes / (dec_avg_ms / 1e3) / 1e9
+    kernel = "decode_tc_kernel" if path == "tcgen05" else "decode_simt_kernel"
+    traffic = recorded_traffic(kernel, wl.name, source_digest(path))
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline_obj(wl, args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "b": b, "h": h, "g": g, "d": d, "m_max": wl.m_max,
+                       "lens": f"U[{wl.len_lo},{wl.len_hi}] (seed {SEED}+rank), mean {float(lens_np.mean()):.0f}",
+                       "step": "kv_append at row lens-1, then decode over lens", "path": path,
+                       "l2": f"{copies} rotating K/V cache copies ({copies * cache_bytes / 2**20:.0f} MiB) so each "
+                             f"step's rows were evicted by >= 2 other steps' reads",
+                       "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": f"mqa_decode call ({kernel} + merge_kernel), avg of {K} event pairs",
+                         "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": dec_avg_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": E},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+            "append_bytes_per_step": append_algorithmic_bytes(wl),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

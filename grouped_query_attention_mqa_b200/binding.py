@@ -1,0 +1,225 @@
+"""ctypes binding of libmqa (include/mqa.h).
+
+Argument marshalling only: shapes and dtypes of torch tensors are read, their
+device pointers and the current CUDA stream are handed to the C ABI, and a
+non-OK status becomes an ``MqaError``.  Every step of the computation runs in
+the library's CUDA kernels; there is no other implementation behind these
+functions and no fallback — if ``libmqa.so`` is missing they raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmqa.so")
+
+MQA_OK, MQA_ERR_INVALID_ARG, MQA_ERR_UNSUPPORTED, MQA_ERR_CUDA = 0, 1, 2, 3
+MQA_F32, MQA_BF16 = 0, 1
+MQA_FLAG_LEN_CLAMPED, MQA_FLAG_POS_SKIPPED, MQA_FLAG_PIPE_TIMEOUT = 1, 2, 4
+PATHS = {"auto": 0, "simt": 1, "tcgen05": 2}
+MQA_MAX_CTAS = 2048
+
+# Every symbol include/mqa.h declares, with its ctypes signature.
+_c_int, _c_size, _c_ptr, _c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+
+
+class DecodeOptions(ctypes.Structure):
+    _fields_ = [("path", _c_int), ("num_ctas", _c_int)]
+
+
+SIGNATURES = {
+    "mqa_kv_append": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_ptr, _c_ptr]),
+    "mqa_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "mqa_decode": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                            _c_float, _c_int, _c_ptr, _c_size, _c_ptr, _c_ptr]),
+    "mqa_decode_ex": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_float, _c_int, _c_ptr, _c_size, _c_ptr, ctypes.POINTER(DecodeOptions),
+                               _c_ptr]),
+    "mqa_status_string": (ctypes.c_char_p, [_c_int]),
+}
+
+
+class MqaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+_LIB = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmqa.so and declare its signatures.  Raises if it is missing."""
+    global _LIB
+    if _LIB is not None and path == LIB_PATH:
+        return _LIB
+    if not os.path.exists(path):
+        raise RuntimeError(f"libmqa.so not built at {path}; run grouped_query_attention_mqa_b200.build.build()")
+    lib_ = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib_, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _LIB = lib_
+    return lib_
+
+
+def lib():
+    return load_library()
+
+
+def status_string(status: int) -> str:
+    return lib().mqa_status_string(int(status)).decode()
+
+
+def decode_workspace_size(b: int, h: int, g: int, d_v: int) -> int:
+    return int(lib().mqa_decode_workspace_size(b, h, g, d_v))
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return MQA_F32
+    if t.dtype == torch.bfloat16:
+        return MQA_BF16
+    raise TypeError(f"libmqa takes float32 or bfloat16 tensors, got {t.dtype}")
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _check_cuda(*tensors):
+    for t in tensors:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libmqa needs contiguous CUDA tensors")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def kv_append(k_cache, v_cache, k_new, v_new, pos, status_flags=None, stream=None):
+    """Write k_new [b,g,d_k] / v_new [b,g,d_v] at row pos[b] of the caches
+    [b,m_max,g,d] (mqa_kv_append)."""
+    import torch
+    _check_cuda(k_cache, v_cache, k_new, v_new, pos, status_flags)
+    b, m_max, g, d_k = k_cache.shape
+    d_v = v_cache.shape[3]
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    if tuple(v_cache.shape[:3]) != (b, m_max, g) or tuple(k_new.shape) != (b, g, d_k) or \
+            tuple(v_new.shape) != (b, g, d_v) or tuple(pos.shape) != (b,):
+        raise ValueError("kv_append: inconsistent shapes")
+    dt = _dtype_code(k_cache)
+    if any(_dtype_code(t) != dt for t in (v_cache, k_new, v_new)):
+        raise TypeError("kv_append: caches and new rows must share one dtype")
+    st = lib().mqa_kv_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(pos), b, m_max, g, d_k,
+                             d_v, dt, _ptr(status_flags), _stream_handle(stream))
+    if st != MQA_OK:
+        raise MqaError(st, "mqa_kv_append")
+
+
+@dataclass
+class _WsCache:
+    tensor: object = None
+
+
+_ws = _WsCache()
+
+
+def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_flags=None, path="auto",
+           num_ctas=0, stream=None):
+    """o [b,h,d_v] = softmax over rows t < lens[b] of scale·q·K, times V
+    (mqa_decode_ex).  ``workspace`` defaults to a torch-allocated buffer of
+    mqa_decode_workspace_size bytes, kept for reuse."""
+    import torch
+    _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags)
+    b, h, d_k = q.shape
+    _, m_max, g, _ = k_cache.shape
+    d_v = v_cache.shape[3]
+    if lens.dtype != torch.int32 or tuple(lens.shape) != (b,):
+        raise ValueError("lens must be int32 [b]")
+    if tuple(k_cache.shape) != (b, m_max, g, d_k) or tuple(v_cache.shape[:3]) != (b, m_max, g):
+        raise ValueError("decode: inconsistent cache shapes")
+    dt = _dtype_code(q)
+    if any(_dtype_code(t) != dt for t in (k_cache, v_cache)):
+        raise TypeError("decode: q and caches must share one dtype")
+    if out is None:
+        out = torch.empty((b, h, d_v), dtype=q.dtype, device=q.device)
+    elif tuple(out.shape) != (b, h, d_v) or out.dtype != q.dtype:
+        raise ValueError("decode: out must be [b,h,d_v] in q's dtype")
+    need = decode_workspace_size(b, h, g, d_v)
+    if workspace is None:
+        ws = _ws.tensor
+        if ws is None or ws.numel() < need or ws.device != q.device:
+            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+            _ws.tensor = ws
+        workspace = ws
+    opts = DecodeOptions(PATHS[path], int(num_ctas))
+    st = lib().mqa_decode_ex(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), b, h, g, m_max, d_k, d_v,
+                             float(scale), dt, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _ptr(status_flags), ctypes.byref(opts), _stream_handle(stream))
+    if st != MQA_OK:
+        raise MqaError(st, "mqa_decode")
+    return out
+
+
+class AppendPlan:
+    """mqa_kv_append with its arguments marshalled once, for loops that repeat
+    the same call (a decode step on fixed buffers): ``run()`` is one C call."""
+
+    def __init__(self, k_cache, v_cache, k_new, v_new, pos, status_flags=None, stream=None):
+        import torch
+        _check_cuda(k_cache, v_cache, k_new, v_new, pos, status_flags)
+        b, m_max, g, d_k = k_cache.shape
+        d_v = v_cache.shape[3]
+        if pos.dtype != torch.int32 or tuple(k_new.shape) != (b, g, d_k) or tuple(v_new.shape) != (b, g, d_v):
+            raise ValueError("AppendPlan: inconsistent arguments")
+        self._keep = (k_cache, v_cache, k_new, v_new, pos, status_flags)
+        self._fn = lib().mqa_kv_append
+        self._args = (_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(pos), b, m_max, g, d_k, d_v,
+                      _dtype_code(k_cache), _ptr(status_flags), _stream_handle(stream))
+
+    def run(self):
+        st = self._fn(*self._args)
+        if st != MQA_OK:
+            raise MqaError(st, "mqa_kv_append")
+
+
+class DecodePlan:
+    """mqa_decode_ex with its arguments marshalled once; ``run()`` is one C call
+    that writes ``self.out``."""
+
+    def __init__(self, q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_flags=None, path="auto",
+                 num_ctas=0, stream=None):
+        import torch
+        _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags)
+        b, h, d_k = q.shape
+        _, m_max, g, _ = k_cache.shape
+        d_v = v_cache.shape[3]
+        if out is None:
+            out = torch.empty((b, h, d_v), dtype=q.dtype, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(max(256, decode_workspace_size(b, h, g, d_v)), dtype=torch.uint8,
+                                    device=q.device)
+        self.out = out
+        self._opts = DecodeOptions(PATHS[path], int(num_ctas))
+        self._keep = (q, k_cache, v_cache, lens, out, workspace, status_flags)
+        self._fn = lib().mqa_decode_ex
+        self._args = (_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), b, h, g, m_max, d_k, d_v,
+                      ctypes.c_float(scale), _dtype_code(q), _ptr(workspace),
+                      workspace.numel() * workspace.element_size(), _ptr(status_flags), ctypes.byref(self._opts),
+                      _stream_handle(stream))
+
+    def run(self):
+        st = self._fn(*self._args)
+        if st != MQA_OK:
+            raise MqaError(st, "mqa_decode")
+        return self.out

@@ -1,0 +1,357 @@
+// Split-KV decode attention on CUDA cores (FFMA), for any element type and
+// small query-head groups.
+//
+// Computation ("Fast Transformer Decoding", velog paper review §3 and §2.4):
+// for each sequence b and K/V head j, the h/g query heads of the group attend
+// over the rows t < L_b of that head's cache,
+//   s_{i,t} = scale * q_i . K_t,  w = softmax_t(s),  o_i = sum_t w_{i,t} V_t.
+// The logits never leave the SM: each tile of TILE rows is staged once in
+// shared memory with cp.async (double buffered, 16-byte copies), every query
+// head of the group reads it from there (the MQA point: one K/V read serves
+// all heads of the group), and an online softmax keeps a running max m and sum
+// l per head.  Exponentials are exp2 of log2(e)-prescaled logits.
+//
+// This path is meant for h/g * d small enough that the arithmetic per byte
+// stays under the FFMA roofline (MHA is 1 FLOP/byte in bf16); larger groups
+// in bf16 go to the tensor-core kernel.
+#include "common.cuh"
+
+namespace mqa {
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTile = 64;
+constexpr int kMaxOutPairs = 16;   // column pairs per thread: h/g * d <= 4096
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+template <typename T, int D>
+struct SimtLayout {
+  static constexpr int kRowBytes = D * int(sizeof(T)) + 16;   // +16: rows land on rotating banks
+  static constexpr int kChunks = D * int(sizeof(T)) / 16;     // 16-byte pieces per row
+  static constexpr int kRedBytes = ((kThreads / 32 + kThreads + 2) * 8 + 15) / 16 * 16;
+  static __host__ __device__ size_t bytes(int hq) {
+    return size_t(kRedBytes) + size_t(hq) * D * 4 + size_t(hq) * kTile * 4 + (size_t(3 * hq) * 4 + 15) / 16 * 16 +
+           size_t(4) * kTile * kRowBytes;
+  }
+};
+
+template <typename T, int D>
+__device__ __forceinline__ void load_tile(unsigned char* ks, unsigned char* vs, const T* __restrict__ K,
+                                          const T* __restrict__ V, const TileCoord& tc, int g, int m_max) {
+  using L = SimtLayout<T, D>;
+  const int n = tc.rows * L::kChunks;
+  const int64_t row_base = (int64_t(tc.seq) * m_max + tc.row0) * g + tc.head;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const int r = i / L::kChunks, c = i - r * L::kChunks;
+    const int64_t off = (row_base + int64_t(r) * g) * D;        // element offset of the row
+    cp_async16(ks + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(K + off) + c * 16);
+    cp_async16(vs + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(V + off) + c * 16);
+  }
+}
+
+// Dot product of a prescaled query (fp32, shared) with `n` elements of a staged
+// row, 16 bytes at a time.
+template <typename T>
+__device__ __forceinline__ float dot_row(const float* __restrict__ q, const unsigned char* row, int e0, int n);
+
+template <>
+__device__ __forceinline__ float dot_row<__nv_bfloat16>(const float* __restrict__ q, const unsigned char* row,
+                                                         int e0, int n) {
+  float acc = 0.f;
+  for (int e = e0; e < e0 + n; e += 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + e * 2);
+    const float4 qa = *reinterpret_cast<const float4*>(q + e);
+    const float4 qb = *reinterpret_cast<const float4*>(q + e + 4);
+    float2 k0 = bf16x2_to_f32x2(w.x), k1 = bf16x2_to_f32x2(w.y), k2 = bf16x2_to_f32x2(w.z),
+           k3 = bf16x2_to_f32x2(w.w);
+    acc = fmaf(qa.x, k0.x, acc);
+    acc = fmaf(qa.y, k0.y, acc);
+    acc = fmaf(qa.z, k1.x, acc);
+    acc = fmaf(qa.w, k1.y, acc);
+    acc = fmaf(qb.x, k2.x, acc);
+    acc = fmaf(qb.y, k2.y, acc);
+    acc = fmaf(qb.z, k3.x, acc);
+    acc = fmaf(qb.w, k3.y, acc);
+  }
+  return acc;
+}
+
+template <>
+__device__ __forceinline__ float dot_row<float>(const float* __restrict__ q, const unsigned char* row, int e0,
+                                                int n) {
+  float acc = 0.f;
+  for (int e = e0; e < e0 + n; e += 4) {
+    const float4 k = *reinterpret_cast<const float4*>(row + e * 4);
+    const float4 qa = *reinterpret_cast<const float4*>(q + e);
+    acc = fmaf(qa.x, k.x, acc);
+    acc = fmaf(qa.y, k.y, acc);
+    acc = fmaf(qa.z, k.z, acc);
+    acc = fmaf(qa.w, k.w, acc);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ float2 load_v_pair(const unsigned char* row, int c2, __nv_bfloat16*) {
+  return bf16x2_to_f32x2(*reinterpret_cast<const uint32_t*>(row + c2 * 4));
+}
+__device__ __forceinline__ float2 load_v_pair(const unsigned char* row, int c2, float*) {
+  return *reinterpret_cast<const float2*>(row + c2 * 8);
+}
+
+__device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
+__device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs a) {
+  using L = SimtLayout<T, D>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  int64_t* red = reinterpret_cast<int64_t*>(smem);
+  float* q_s = reinterpret_cast<float*>(smem + L::kRedBytes);
+  float* p_s = q_s + a.hq * D;
+  float* m_s = p_s + a.hq * kTile;
+  float* l_s = m_s + a.hq;
+  float* al_s = l_s + a.hq;
+  unsigned char* stage = reinterpret_cast<unsigned char*>(m_s) + (size_t(3 * a.hq) * 4 + 15) / 16 * 16;
+  // stage s: K at stage + s*kStageBytes, V at stage + (2+s)*kStageBytes
+  constexpr int kStageBytes = kTile * L::kRowBytes;
+
+  const T* __restrict__ Q = static_cast<const T*>(a.q);
+  const T* __restrict__ K = static_cast<const T*>(a.k);
+  const T* __restrict__ V = static_cast<const T*>(a.v);
+  T* __restrict__ O = static_cast<T*>(a.o);
+  const int hq = a.hq, g = a.g;
+  const float qscale = a.scale * kLog2e;
+
+  // Inputs may come from the kernel before this one on the stream (the append).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const Sched sc = make_schedule<kThreads>(a.lens, a.b, g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, red);
+  if (sc.t_begin >= sc.t_end) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    return;
+  }
+
+  Cursor cur = cursor_at(a.lens, a.m_max, kTile, sc.seq, sc.seq_base);
+  Cursor nxt = cur;
+  cursor_seek(cur, a.lens, g, a.m_max, kTile, sc.t_begin);
+  {
+    const TileCoord t0 = tile_coord(cur, g, kTile, sc.t_begin);
+    load_tile<T, D>(stage, stage + 2 * kStageBytes, K, V, t0, g, a.m_max);
+    cp_async_commit();
+  }
+
+  const int pairs_out = hq * (D / 2);
+  float2 acc[kMaxOutPairs];
+#pragma unroll
+  for (int r = 0; r < kMaxOutPairs; ++r) acc[r] = make_float2(0.f, 0.f);
+
+  const int lg_pairs = hq * kTile;
+  const int split = lg_pairs < kThreads ? kThreads / lg_pairs : 1;   // threads per (head, row)
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  for (int64_t t = sc.t_begin; t < sc.t_end; ++t) {
+    const int st = int((t - sc.t_begin) & 1);
+    cursor_seek(cur, a.lens, g, a.m_max, kTile, t);
+    const TileCoord tc = tile_coord(cur, g, kTile, t);
+
+    if (t == sc.t_begin || tc.k == 0) {   // a new segment starts: its queries, fresh state
+      const T* qg = Q + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq) * D;
+      for (int i = threadIdx.x; i < hq * D; i += kThreads) q_s[i] = to_f32(qg[i]) * qscale;
+      for (int i = threadIdx.x; i < hq; i += kThreads) {
+        m_s[i] = -INFINITY;
+        l_s[i] = 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxOutPairs; ++r) acc[r] = make_float2(0.f, 0.f);
+    }
+    if (t + 1 < sc.t_end) {
+      cursor_seek(nxt, a.lens, g, a.m_max, kTile, t + 1);
+      const TileCoord tn = tile_coord(nxt, g, kTile, t + 1);
+      load_tile<T, D>(stage + (st ^ 1) * kStageBytes, stage + (2 + (st ^ 1)) * kStageBytes, K, V, tn, g,
+                      a.m_max);
+    }
+    cp_async_commit();
+    cp_async_wait1();
+    __syncthreads();
+
+    // logits, prescaled by scale*log2(e); rows past the valid count are -inf
+    for (int p = threadIdx.x / split; p < lg_pairs; p += kThreads / split) {
+      const int i = p / kTile, r = p - i * kTile;
+      const int part = threadIdx.x % split;
+      float s = 0.f;
+      if (r < tc.rows) s = dot_row<T>(q_s + i * D, stage + st * kStageBytes + r * L::kRowBytes, part * (D / split), D / split);
+      for (int o = split / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (part == 0) p_s[i * kTile + r] = r < tc.rows ? s : -INFINITY;
+    }
+    __syncthreads();
+
+    // online softmax, one warp per head
+    for (int i = warp; i < hq; i += kThreads / 32) {
+      const float s0 = p_s[i * kTile + lane], s1 = p_s[i * kTile + lane + 32];
+      float mx = fmaxf(s0, s1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_old = m_s[i];
+      const float m_new = fmaxf(m_old, mx);
+      const float p0 = exp2f(s0 - m_new), p1 = exp2f(s1 - m_new);
+      p_s[i * kTile + lane] = p0;
+      p_s[i * kTile + lane + 32] = p1;
+      float sum = p0 + p1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) {
+        const float alpha = exp2f(m_old - m_new);
+        al_s[i] = alpha;
+        l_s[i] = l_s[i] * alpha + sum;
+        m_s[i] = m_new;
+      }
+    }
+    __syncthreads();
+
+    // weighted V: thread owns column pairs (head i, columns 2c2, 2c2+1)
+#pragma unroll
+    for (int r = 0; r < kMaxOutPairs; ++r) {
+      const int f = threadIdx.x + r * kThreads;
+      if (f < pairs_out) {
+        const int i = f / (D / 2), c2 = f - i * (D / 2);
+        const float alpha = al_s[i];
+        float2 o2 = make_float2(acc[r].x * alpha, acc[r].y * alpha);
+        const float* pw = p_s + i * kTile;
+        const unsigned char* vrow = stage + (2 + st) * kStageBytes;
+        for (int row = 0; row < tc.rows; ++row) {
+          const float w = pw[row];
+          const float2 v = load_v_pair(vrow + row * L::kRowBytes, c2, static_cast<T*>(nullptr));
+          o2.x = fmaf(w, v.x, o2.x);
+          o2.y = fmaf(w, v.y, o2.y);
+        }
+        acc[r] = o2;
+      }
+    }
+
+    const bool seg_last = (tc.k == tc.nb - 1) || (t + 1 == sc.t_end);
+    if (seg_last) {
+      const bool owns_first = tc.seg_t0 >= sc.t_begin;
+      const bool whole = owns_first && (tc.seg_t0 + tc.nb <= sc.t_end);
+      const int64_t slot = partial_slot(blockIdx.x, tc.seg);
+#pragma unroll
+      for (int r = 0; r < kMaxOutPairs; ++r) {
+        const int f = threadIdx.x + r * kThreads;
+        if (f < pairs_out) {
+          const int i = f / (D / 2), c2 = f - i * (D / 2);
+          const float inv = 1.f / l_s[i];
+          const float2 v = make_float2(acc[r].x * inv, acc[r].y * inv);
+          if (whole) {
+            store_pair(O + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq + i) * D + 2 * c2, v);
+          } else {
+            *reinterpret_cast<float2*>(a.ws.part_o + (slot * hq + i) * D + 2 * c2) = v;
+          }
+        }
+      }
+      if (!whole)
+        for (int i = threadIdx.x; i < hq; i += kThreads) a.ws.part_lse[slot * hq + i] = m_s[i] + log2f(l_s[i]);
+      if (owns_first && threadIdx.x == 0)
+        a.ws.seg_info[tc.seg] =
+            make_int2(blockIdx.x, cta_of_tile(tc.seg_t0 + tc.nb - 1, sc.total, sc.active));
+    }
+    __syncthreads();
+  }
+  asm volatile("griddepcontrol.launch_dependents;");
+}
+
+// Opt the kernel into large dynamic shared memory once per device.
+template <typename T, int D>
+cudaError_t ensure_smem_attr() {
+  static bool done[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_simt_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
+  const size_t smem = SimtLayout<T, D>::bytes(a.hq);
+  cudaError_t e = ensure_smem_attr<T, D>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(a.grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_simt_kernel<T, D>, a);
+}
+
+// Resident CTAs per SM for this shared-memory size, cached per (device, h/g).
+template <typename T, int D>
+int occupancy_t(int hq) {
+  static int cache[64][129] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  const bool cacheable = dev >= 0 && dev < 64 && hq >= 1 && hq <= 128;
+  if (cacheable && cache[dev][hq] > 0) return cache[dev][hq];
+  const size_t smem = SimtLayout<T, D>::bytes(hq);
+  if (ensure_smem_attr<T, D>() != cudaSuccess) return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_simt_kernel<T, D>, kThreads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  if (cacheable) cache[dev][hq] = n;
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream) {
+  if (dtype == MQA_BF16) {
+    switch (a.d) {
+      case 32: return launch_t<__nv_bfloat16, 32>(a, stream);
+      case 64: return launch_t<__nv_bfloat16, 64>(a, stream);
+      case 128: return launch_t<__nv_bfloat16, 128>(a, stream);
+    }
+  } else {
+    switch (a.d) {
+      case 32: return launch_t<float, 32>(a, stream);
+      case 64: return launch_t<float, 64>(a, stream);
+      case 128: return launch_t<float, 128>(a, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq) {
+  if (dtype == MQA_BF16) {
+    switch (d) {
+      case 32: return occupancy_t<__nv_bfloat16, 32>(hq);
+      case 64: return occupancy_t<__nv_bfloat16, 64>(hq);
+      case 128: return occupancy_t<__nv_bfloat16, 128>(hq);
+    }
+  } else {
+    switch (d) {
+      case 32: return occupancy_t<float, 32>(hq);
+      case 64: return occupancy_t<float, 64>(hq);
+      case 128: return occupancy_t<float, 128>(hq);
+    }
+  }
+  return 1;
+}
+
+}  // namespace mqa

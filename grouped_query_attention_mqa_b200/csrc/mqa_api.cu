@@ -1,0 +1,135 @@
+// The C ABI of libmqa: argument checks, the choice of kernel path and CTA
+// count, and the launches.  No allocation, no synchronisation, no exceptions.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace {
+
+using namespace mqa;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+int elem_bytes(mqa_dtype_t dt) { return dt == MQA_F32 ? 4 : 2; }
+bool valid_dtype(int dt) { return dt == MQA_F32 || dt == MQA_BF16; }
+
+// SM count of the current device, cached per device.
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mqa_status_string(mqa_status_t s) {
+  switch (s) {
+    case MQA_OK: return "MQA_OK";
+    case MQA_ERR_INVALID_ARG: return "MQA_ERR_INVALID_ARG";
+    case MQA_ERR_UNSUPPORTED: return "MQA_ERR_UNSUPPORTED";
+    case MQA_ERR_CUDA: return "MQA_ERR_CUDA";
+  }
+  return "MQA_STATUS_UNKNOWN";
+}
+
+mqa_status_t mqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos,
+                           int b, int m_max, int g, int d_k, int d_v, mqa_dtype_t dtype, int32_t* status_flags,
+                           cudaStream_t stream) {
+  if (b < 0 || m_max < 1 || g < 1 || d_k < 1 || d_v < 1 || !valid_dtype(dtype)) return MQA_ERR_INVALID_ARG;
+  if (b == 0) return MQA_OK;
+  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return MQA_ERR_INVALID_ARG;
+  const int64_t row_k = int64_t(g) * d_k * elem_bytes(dtype), row_v = int64_t(g) * d_v * elem_bytes(dtype);
+  if (row_k % 16 != 0 || row_v % 16 != 0 || row_k > (int64_t(1) << 30) || row_v > (int64_t(1) << 30))
+    return MQA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(pos))
+    return MQA_ERR_INVALID_ARG;
+  if (launch_append(k_cache, v_cache, k_new, v_new, pos, b, m_max, g, int(row_k), int(row_v), status_flags,
+                    stream) != cudaSuccess)
+    return MQA_ERR_CUDA;
+  return MQA_OK;
+}
+
+size_t mqa_decode_workspace_size(int b, int h, int g, int d_v) {
+  if (b < 0 || h < 1 || g < 1 || h % g != 0 || d_v < 1) return 0;
+  return workspace_bytes(b, g, h / g, d_v);
+}
+
+mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens,
+                           int b, int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes_given, int32_t* status_flags,
+                           const mqa_decode_opts_t* opts, cudaStream_t stream) {
+  if (b < 0 || h < 1 || g < 1 || h % g != 0 || m_max < 1 || d_k < 1 || d_v < 1 || !valid_dtype(dtype) ||
+      !std::isfinite(scale))
+    return MQA_ERR_INVALID_ARG;
+  const int path = opts ? opts->path : MQA_PATH_AUTO;
+  if (path < MQA_PATH_AUTO || path > MQA_PATH_TCGEN05) return MQA_ERR_INVALID_ARG;
+  if (opts && (opts->num_ctas < 0 || opts->num_ctas > kMaxCtas)) return MQA_ERR_INVALID_ARG;
+  if (b == 0) return MQA_OK;
+  if (!o || !q || !k_cache || !v_cache || !lens || !workspace) return MQA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(lens) ||
+      !aligned256(workspace))
+    return MQA_ERR_INVALID_ARG;
+  if (int64_t(b) * g > (int64_t(1) << 30) || int64_t(b) * m_max * g > (int64_t(1) << 40))
+    return MQA_ERR_INVALID_ARG;
+  const int hq = h / g;
+  if (workspace_bytes_given < workspace_bytes(b, g, hq, d_v)) return MQA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 32 && d_k != 64 && d_k != 128)) return MQA_ERR_UNSUPPORTED;
+
+  const bool tc_ok = dtype == MQA_BF16 && tc_supported(d_k, hq);
+  const bool simt_ok = int64_t(hq) * d_k <= 4096;
+  bool use_tc;
+  if (path == MQA_PATH_TCGEN05) {
+    if (!tc_ok) return MQA_ERR_UNSUPPORTED;
+    use_tc = true;
+  } else if (path == MQA_PATH_SIMT) {
+    if (!simt_ok) return MQA_ERR_UNSUPPORTED;
+    use_tc = false;
+  } else {
+    use_tc = tc_ok && hq >= 8;
+    if (!use_tc && !simt_ok) return MQA_ERR_UNSUPPORTED;
+  }
+
+  const int sms = sm_count();
+  if (sms <= 0) return MQA_ERR_CUDA;
+  DecodeArgs a;
+  a.o = o;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.lens = lens;
+  a.b = b;
+  a.h = h;
+  a.g = g;
+  a.m_max = m_max;
+  a.d = d_k;
+  a.hq = hq;
+  a.scale = scale;
+  a.ws = carve_workspace(workspace, b, g, hq);
+  a.flags = status_flags;
+  int grid = opts && opts->num_ctas > 0 ? opts->num_ctas
+                                         : sms * (use_tc ? tc_ctas_per_sm(hq) : simt_ctas_per_sm(dtype, d_k, hq));
+  a.grid = grid < 1 ? 1 : (grid > kMaxCtas ? kMaxCtas : grid);
+
+  cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, dtype, stream);
+  if (e != cudaSuccess) return MQA_ERR_CUDA;
+  e = launch_merge(a, dtype, stream);
+  if (e != cudaSuccess) return MQA_ERR_CUDA;
+  return MQA_OK;
+}
+
+mqa_status_t mqa_decode(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int b,
+                        int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype, void* workspace,
+                        size_t workspace_bytes_given, int32_t* status_flags, cudaStream_t stream) {
+  return mqa_decode_ex(o, q, k_cache, v_cache, lens, b, h, g, m_max, d_k, d_v, scale, dtype, workspace,
+                       workspace_bytes_given, status_flags, nullptr, stream);
+}
+
+}  // extern "C"

@@ -26,15 +26,26 @@ BF16_NAN_BITS = 0x7FC0
 
 def f32_to_bf16_bits(x):
     """float32 array -> bf16 bit patterns (uint16), round to nearest even.
-    NaN stays NaN (quiet)."""
+    NaN stays NaN (quiet).  Works in fixed-size chunks with reused buffers so
+    multi-GB caches do not allocate GB-sized temporaries."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    out = rounded.astype(np.uint16)
-    nan = np.isnan(x)
-    if nan.any():
-        out[nan] = BF16_NAN_BITS
-    return out
+    u = x.reshape(-1).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    chunk = 1 << 22
+    tmp = np.empty(min(chunk, u.size), dtype=np.uint32)
+    for s in range(0, u.size, chunk):
+        e = min(u.size, s + chunk)
+        t = tmp[: e - s]
+        np.right_shift(u[s:e], 16, out=t)
+        np.bitwise_and(t, 1, out=t)
+        np.add(t, u[s:e], out=t)
+        np.add(t, 0x7FFF, out=t)          # no wrap: the largest non-NaN pattern is 0xFF800000
+        np.right_shift(t, 16, out=t)
+        out[s:e] = t
+        nan = np.isnan(x.reshape(-1)[s:e])
+        if nan.any():
+            out[s:e][nan] = BF16_NAN_BITS
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(bits):

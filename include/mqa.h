@@ -1,0 +1,170 @@
+/*
+ * libmqa — single-token incremental-decode attention over a KV cache, for
+ * NVIDIA B200 (sm_100a).  Multi-Query Attention (h query heads share one K/V
+ * head), Grouped-Query Attention (g K/V heads, each shared by h/g query heads)
+ * and Multi-Head Attention (g = h) are one computation with one parameter g.
+ *
+ * The computation, from the incremental decode step of "Fast Transformer
+ * Decoding: One Write-Head is All You Need" (the velog paper review, §3
+ * "Multi Query Attention", MultiquerySelfAttentionIncremental; §2.4 for the
+ * per-head MHA form) with the projections left to the caller:
+ *
+ *   new_K = concat(prev_K, k_new)                       -> mqa_kv_append
+ *   logits = einsum("bhk,bmk->bhm", q, new_K) * scale   -> mqa_decode
+ *   weights = softmax(logits) over each sequence's valid rows
+ *   o = einsum("bhm,bmv->bhv", weights, new_V)
+ *
+ * Grouping follows the GQA blog ("GQA、MQA、MLA", section "第三站: GQA"):
+ * query head i reads K/V head j = i / (h/g).  The scale is the 1/sqrt(d_h) of
+ * the study notes' §1 formula when the caller wants it; pass 1.0 when q is
+ * already scaled (the paper's code has no scale).
+ *
+ * Conventions shared by every call
+ *  - All pointers named "device" are CUDA device pointers on the current
+ *    device, owned by the caller, 16-byte aligned, and not aliased with each
+ *    other.  The library allocates nothing and keeps no state between calls
+ *    besides per-device attribute caches.
+ *  - Tensors are dense and row-major in the stated shapes.  q, the caches and
+ *    o share one element type (mqa_dtype_t); arithmetic is fp32 throughout.
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ *    Arguments are checked before anything is launched: a failed check
+ *    returns MQA_ERR_INVALID_ARG or MQA_ERR_UNSUPPORTED and launches nothing.
+ *    A launch failure returns MQA_ERR_CUDA.  Nothing traps, nothing throws.
+ *  - Values read on the device (lens, pos) are clamped or skipped, never
+ *    trusted: the offending case sets a bit in *status_flags (a caller-owned
+ *    device int32, may be NULL) with an atomic OR.  The library never clears
+ *    it; the caller zeroes it when it wants a fresh reading.
+ */
+#ifndef LIBMQA_MQA_H
+#define LIBMQA_MQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MQA_API __attribute__((visibility("default")))
+#else
+#define MQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MQA_OK = 0,
+  MQA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or combination */
+  MQA_ERR_UNSUPPORTED = 2,   /* valid, but not built (e.g. head size 96)      */
+  MQA_ERR_CUDA = 3           /* a CUDA call or launch failed                  */
+} mqa_status_t;
+
+typedef enum {
+  MQA_F32 = 0,               /* float32 storage                                */
+  MQA_BF16 = 1               /* bfloat16 storage, round-to-nearest-even output */
+} mqa_dtype_t;
+
+/* Bits of *status_flags. */
+#define MQA_FLAG_LEN_CLAMPED 1 /* a lens[b] was outside [1, m_max]; clamped     */
+#define MQA_FLAG_POS_SKIPPED 2 /* a pos[b] was outside [0, m_max); not written  */
+#define MQA_FLAG_PIPE_TIMEOUT 4 /* a tensor-core pipeline wait ran out; the
+                                   outputs of that call are not valid           */
+
+/* Kernel path of mqa_decode_ex. */
+typedef enum {
+  MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d = 128 and h/g >= 8  */
+  MQA_PATH_SIMT = 1,         /* CUDA-core FFMA path (any dtype, h/g*d <= 4096) */
+  MQA_PATH_TCGEN05 = 2       /* tcgen05 tensor-core path (bf16, d = 128,
+                                8 <= h/g <= 128)                              */
+} mqa_path_t;
+
+typedef struct {
+  int path;                  /* mqa_path_t                                     */
+  int num_ctas;              /* persistent CTAs; 0 = SM count x resident CTAs  */
+} mqa_decode_opts_t;
+
+/* Largest number of persistent CTAs a decode may use; sizes the workspace. */
+#define MQA_MAX_CTAS 2048
+
+/*
+ * mqa_kv_append — write one step's K and V into the cache ("one write-head").
+ *
+ * Source: the velog paper review, §3 MultiquerySelfAttentionIncremental,
+ * new_K = concat([prev_K, expand_dims(k_new)]) and the same for V; with a
+ * fixed-size cache the concat is a write at row pos[b].
+ *
+ *   k_cache  device [b, m_max, g, d_k]   written at rows pos[b] only
+ *   v_cache  device [b, m_max, g, d_v]   written at rows pos[b] only
+ *   k_new    device [b, g, d_k]          read
+ *   v_new    device [b, g, d_v]          read
+ *   pos      device int32 [b]            row to write for each sequence
+ *   status_flags  device int32 or NULL   MQA_FLAG_POS_SKIPPED when some pos[b]
+ *                                        is outside [0, m_max); that sequence
+ *                                        is left untouched
+ * The copy is bitwise.  b = 0 is a no-op returning MQA_OK.  Errors:
+ * MQA_ERR_INVALID_ARG for NULL pointers, negative sizes, a row size
+ * (d * element size) that is not a multiple of 16 bytes, or misalignment.
+ * Intended order within a step: append at pos = old length, then decode with
+ * lens = old length + 1 (the review's step concatenates before attending).
+ */
+MQA_API mqa_status_t mqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                           const int32_t* pos, int b, int m_max, int g, int d_k, int d_v,
+                           mqa_dtype_t dtype, int32_t* status_flags, cudaStream_t stream);
+
+/*
+ * mqa_decode_workspace_size — bytes of device scratch mqa_decode needs.
+ * Pure host arithmetic (no CUDA call).  The workspace holds, per split of a
+ * sequence's rows, the normalised partial output (fp32 [h/g, d_v]) and its
+ * log-sum-exp, plus two ints per (sequence, K/V head).  Returns 0 for
+ * invalid sizes.
+ */
+MQA_API size_t mqa_decode_workspace_size(int b, int h, int g, int d_v);
+
+/*
+ * mqa_decode — attention of each sequence's newest query over its cache.
+ *
+ * Source: the velog paper review, §3 (MQA) and §2.4 (MHA) incremental code,
+ * logits = einsum("bhk,bmk->bhm"), softmax, o = einsum("bhm,bmv->bhv"); the
+ * scaled softmax of the study notes §1; GQA grouping of the GQA blog.
+ *
+ *   o        device [b, h, d_v]          written (every element)
+ *   q        device [b, h, d_k]          read
+ *   k_cache  device [b, m_max, g, d_k]   rows t < lens[b] read; others never
+ *   v_cache  device [b, m_max, g, d_v]   rows t < lens[b] read; others never
+ *   lens     device int32 [b]            valid rows per sequence; values
+ *                                        outside [1, m_max] are clamped
+ *                                        (<= 0 gives an all-zero output row)
+ *                                        and set MQA_FLAG_LEN_CLAMPED
+ *   scale    multiplies q . k (finite)
+ *   workspace        device scratch of at least
+ *                    mqa_decode_workspace_size(b, h, g, d_v) bytes, 256-byte
+ *                    aligned; contents on entry do not matter; calls that
+ *                    share a workspace must be ordered on one stream
+ *   status_flags     device int32 or NULL (see above)
+ * Supported: h % g == 0, d_k == d_v in {32, 64, 128}, and h/g * d_v <= 4096
+ * on the SIMT path.  b = 0 is a no-op returning MQA_OK.
+ * Errors: MQA_ERR_INVALID_ARG (NULL pointer, h % g != 0, non-finite scale,
+ * workspace too small or misaligned), MQA_ERR_UNSUPPORTED (head sizes or
+ * group widths not built), MQA_ERR_CUDA (launch failure).
+ */
+MQA_API mqa_status_t mqa_decode(void* o, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* lens, int b, int h, int g, int m_max, int d_k, int d_v,
+                        float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                        int32_t* status_flags, cudaStream_t stream);
+
+/* mqa_decode with an explicit kernel path and CTA count (opts may be NULL,
+ * which is mqa_decode).  Requesting a path that cannot serve the arguments
+ * returns MQA_ERR_UNSUPPORTED. */
+MQA_API mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* lens, int b, int h, int g, int m_max, int d_k, int d_v,
+                           float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                           int32_t* status_flags, const mqa_decode_opts_t* opts, cudaStream_t stream);
+
+/* Static, NUL-terminated name of a status code. */
+MQA_API const char* mqa_status_string(mqa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBMQA_MQA_H */

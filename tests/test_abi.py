@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: the library builds and loads, exports every symbol
+include/mqa.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_query_attention_mqa_b200 import binding
+from grouped_query_attention_mqa_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "mqa.h")).read()
+    return sorted(set(re.findall(r"MQA_API\s+[\w\s\*]+?\b(mqa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert header_symbols() == sorted(["mqa_kv_append", "mqa_decode_workspace_size", "mqa_decode",
+                                       "mqa_decode_ex", "mqa_status_string"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+    assert set(header_symbols()) == set(binding.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert binding.status_string(0) == "MQA_OK"
+    assert binding.status_string(1) == "MQA_ERR_INVALID_ARG"
+    assert binding.status_string(2) == "MQA_ERR_UNSUPPORTED"
+    assert binding.status_string(3) == "MQA_ERR_CUDA"
+    assert binding.status_string(99) == "MQA_STATUS_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    ws = binding.decode_workspace_size
+    assert ws(64, 32, 1, 128) > 0
+    # grows with the batch and the group width
+    assert ws(128, 32, 1, 128) > ws(64, 32, 1, 128)
+    assert ws(64, 64, 1, 128) > ws(64, 32, 1, 128)
+    # partial slots: one per persistent CTA plus one per (sequence, K/V head)
+    slots = binding.MQA_MAX_CTAS + 64
+    assert ws(64, 32, 1, 128) >= slots * 32 * 129 * 4
+    for bad in ((64, 32, 3, 128), (-1, 8, 1, 128), (4, 0, 1, 128), (4, 8, 0, 128), (4, 8, 1, 0)):
+        assert ws(*bad) == 0
+    assert ws(0, 8, 1, 128) > 0   # empty batch: only the per-CTA slots
+
+
+FAKE = ctypes.c_void_p(0x10000)   # aligned, never dereferenced: every call below fails its checks first
+
+
+def _decode(lib, **kw):
+    a = dict(o=FAKE, q=FAKE, k=FAKE, v=FAKE, lens=FAKE, b=2, h=8, g=1, m_max=16, d_k=128, d_v=128, scale=1.0,
+             dtype=binding.MQA_BF16, ws=FAKE, ws_bytes=1 << 40, flags=None, opts=None, stream=None)
+    a.update(kw)
+    return lib.mqa_decode_ex(a["o"], a["q"], a["k"], a["v"], a["lens"], a["b"], a["h"], a["g"], a["m_max"],
+                             a["d_k"], a["d_v"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"], a["flags"],
+                             a["opts"], a["stream"])
+
+
+def test_decode_rejects_bad_arguments_without_launching(lib):
+    INV, UNS = binding.MQA_ERR_INVALID_ARG, binding.MQA_ERR_UNSUPPORTED
+    assert _decode(lib, g=3) == INV                      # h % g != 0
+    assert _decode(lib, g=0) == INV
+    assert _decode(lib, q=None) == INV
+    assert _decode(lib, ws=None) == INV
+    assert _decode(lib, o=ctypes.c_void_p(0x10008)) == INV        # misaligned
+    assert _decode(lib, ws=ctypes.c_void_p(0x10010)) == INV       # workspace not 256-aligned
+    assert _decode(lib, ws_bytes=100) == INV             # workspace too small
+    assert _decode(lib, scale=float("nan")) == INV
+    assert _decode(lib, scale=float("inf")) == INV
+    assert _decode(lib, dtype=7) == INV
+    assert _decode(lib, m_max=0) == INV
+    assert _decode(lib, d_k=96, d_v=96) == UNS           # head size not built
+    assert _decode(lib, d_k=128, d_v=64) == UNS          # d_k != d_v not built
+    opts = binding.DecodeOptions(9, 0)
+    assert _decode(lib, opts=ctypes.byref(opts)) == INV  # unknown path
+    opts = binding.DecodeOptions(0, binding.MQA_MAX_CTAS + 1)
+    assert _decode(lib, opts=ctypes.byref(opts)) == INV
+    opts = binding.DecodeOptions(1, 0)                   # SIMT cannot take h/g*d > 4096
+    assert _decode(lib, h=64, opts=ctypes.byref(opts)) == UNS
+    opts = binding.DecodeOptions(2, 0)                   # tensor cores need bf16
+    assert _decode(lib, dtype=binding.MQA_F32, opts=ctypes.byref(opts)) == UNS
+    assert _decode(lib, b=0) == binding.MQA_OK           # empty batch: nothing to do
+
+
+def test_append_rejects_bad_arguments_without_launching(lib):
+    INV = binding.MQA_ERR_INVALID_ARG
+    f = lib.mqa_kv_append
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 1, 128, 128, 1, None, None) == INV       # m_max
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 2, 8, 1, 128, 128, 1, None, None) == INV
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 128, 128, 1, None, None) == INV
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 1, 4, 4, 1, None, None) == INV           # 8-byte rows
+    assert f(FAKE, FAKE, ctypes.c_void_p(0x10004), FAKE, FAKE, 2, 8, 1, 128, 128, 1, None, None) == INV
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 1, 128, 128, 5, None, None) == INV       # dtype
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 8, 1, 128, 128, 1, None, None) == INV
+    assert f(None, None, None, None, None, 0, 8, 1, 128, 128, 1, None, None) == binding.MQA_OK
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.load_library(str(tmp_path / "libmqa.so"))
