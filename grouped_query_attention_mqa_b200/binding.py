@@ -20,6 +20,7 @@ MQA_F32, MQA_BF16 = 0, 1
 MQA_FLAG_LEN_CLAMPED, MQA_FLAG_POS_SKIPPED, MQA_FLAG_PIPE_TIMEOUT = 1, 2, 4
 PATHS = {"auto": 0, "simt": 1, "tcgen05": 2}
 MQA_MAX_CTAS = 2048
+MQA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/mqa.h declares, with its ctypes signature.
 _c_int, _c_size, _c_ptr, _c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
@@ -38,6 +39,8 @@ SIGNATURES = {
     "mqa_decode_ex": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_float, _c_int, _c_ptr, _c_size, _c_ptr, ctypes.POINTER(DecodeOptions),
                                _c_ptr]),
+    "mqa_decode_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                    _c_int, _c_float, _c_int, _c_ptr, _c_ptr]),
     "mqa_status_string": (ctypes.c_char_p, [_c_int]),
 }
 

@@ -160,6 +160,44 @@ MQA_API mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, 
                            float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes,
                            int32_t* status_flags, const mqa_decode_opts_t* opts, cudaStream_t stream);
 
+/* Size of the device array that mqa_decode_noalloc uses as its scratch. */
+#define MQA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * mqa_decode_noalloc — mqa_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a deployment variant of
+ * the same computation, not a step of the method.
+ *
+ * Who needs it: code that must not call cudaMalloc or any other allocator —
+ * a plugin whose host application owns all device memory, a runtime with a
+ * memory pool fixed at start-up, or a call site where an allocation could
+ * synchronise the device or fail at a point where failure is not allowed.
+ * Instead of a caller-provided workspace, the split partials live in a
+ * device array of MQA_NOALLOC_SCRATCH_BYTES (16 MiB) that the library
+ * defines; every GPU on which the library is loaded holds that array until
+ * the process exits.  The call allocates nothing.
+ *
+ * Arguments, results, flags and errors are those of mqa_decode without the
+ * workspace pair; the caller still provides o, q, the caches and lens.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current).  Make that first call before any
+ *    stream capture on the device.
+ *  - The array holds the partials of the last call; every value a call reads
+ *    back from it was written earlier in the same call, so nothing in it has
+ *    to start at zero.
+ *  - All calls on a device share the one array: calls whose work can overlap
+ *    on the GPU (different streams without ordering, several host threads)
+ *    race on it and give wrong results.  Order them on one stream.
+ *  - Shapes whose partials cannot fit even with a single CTA (roughly
+ *    b * g * h/g * (d_v + 1) * 4 bytes above 16 MiB) are rejected with
+ *    MQA_ERR_INVALID_ARG before anything is launched; otherwise the number of
+ *    CTAs is lowered until the partials fit.
+ */
+MQA_API mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* lens, int b, int h, int g, int m_max, int d_k, int d_v,
+                                        float scale, mqa_dtype_t dtype, int32_t* status_flags,
+                                        cudaStream_t stream);
+
 /* Static, NUL-terminated name of a status code. */
 MQA_API const char* mqa_status_string(mqa_status_t status);
 
