@@ -75,7 +75,7 @@ typedef enum {
   MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d = 128 and h/g >= 8  */
   MQA_PATH_SIMT = 1,         /* CUDA-core FFMA path (any dtype, h/g*d <= 4096) */
   MQA_PATH_TCGEN05 = 2       /* tcgen05 tensor-core path (bf16, d = 128,
-                                8 <= h/g <= 128)                              */
+                                h/g <= 64)                                    */
 } mqa_path_t;
 
 typedef struct {
@@ -141,8 +141,8 @@ MQA_API size_t mqa_decode_workspace_size(int b, int h, int g, int d_v);
  *                    aligned; contents on entry do not matter; calls that
  *                    share a workspace must be ordered on one stream
  *   status_flags     device int32 or NULL (see above)
- * Supported: h % g == 0, d_k == d_v in {32, 64, 128}, and h/g * d_v <= 4096
- * on the SIMT path.  b = 0 is a no-op returning MQA_OK.
+ * Supported: h % g == 0, d_k == d_v in {32, 64, 128}; the SIMT path takes
+ * h/g * d_v <= 4096, the tensor-core path bf16 with d = 128 and h/g <= 64.  b = 0 is a no-op returning MQA_OK.
  * Errors: MQA_ERR_INVALID_ARG (NULL pointer, h % g != 0, non-finite scale,
  * workspace too small or misaligned), MQA_ERR_UNSUPPORTED (head sizes or
  * group widths not built), MQA_ERR_CUDA (launch failure).

@@ -25,7 +25,7 @@ def _lib():
 
 
 def tc_available(wl):
-    return wl.dtype == "bf16" and wl.d_k == 128 and 8 <= wl.heads_per_group <= 128 and _tc_built()
+    return wl.dtype == "bf16" and wl.d_k == 128 and 1 <= wl.heads_per_group <= 64 and _tc_built()
 
 
 def _tc_built():
@@ -97,7 +97,7 @@ def test_decode_matches_oracle(shape, num_ctas):
 
 
 @pytest.mark.parametrize("path", ["simt", "tcgen05"])
-@pytest.mark.parametrize("hq", [8, 16, 32, 64, 128])
+@pytest.mark.parametrize("hq", [1, 4, 8, 12, 16, 32, 48, 64])
 def test_both_paths_on_group_widths(path, hq):
     wl = small("bf16", 3, hq, 1, 128, 530, 1, 530)
     if path == "tcgen05" and not tc_available(wl):
@@ -107,6 +107,38 @@ def test_both_paths_on_group_widths(path, hq):
     for num_ctas in (0, 2, 5):
         out, ref = run_case(wl, seed=hq + num_ctas, path=path, num_ctas=num_ctas)
         assert_close(out, ref, "bf16", f"{path} hq={hq} ctas={num_ctas}")
+
+
+@pytest.mark.parametrize("g", [1, 2, 8])
+def test_tensor_core_path_gqa_and_tile_edges(g):
+    """The tensor-core path with several K/V heads and lengths at its 128-row
+    tile edges, whole sequences and sequences split between CTAs."""
+    wl = small("bf16", 4, 8 * g, g, 128, 400, 1, 1)
+    if not tc_available(wl):
+        pytest.skip("tensor-core path not built")
+    for lens in ([127, 128, 129, 400], [1, 2, 255, 256], [257, 383, 384, 385]):
+        for num_ctas in (0, 1, 3, 9):
+            out, ref = run_case(wl, seed=sum(lens) + num_ctas, lens=np.array(lens, np.int32), path="tcgen05",
+                                num_ctas=num_ctas)
+            assert_close(out, ref, "bf16", f"tc g={g} lens={lens} ctas={num_ctas}")
+
+
+def test_tensor_core_path_rescales_for_growing_logits():
+    """Logits that grow along the sequence force the running maximum to move
+    (and O in tensor memory to be rescaled) several times within a segment."""
+    wl = small("bf16", 2, 32, 1, 128, 1024, 1024, 1024)
+    if not tc_available(wl):
+        pytest.skip("tensor-core path not built")
+    inp = host_inputs(wl, seed=21, nan_tail=True)
+    from grouped_query_attention_mqa_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits
+    ramp = np.linspace(0.0, 6.0, wl.m_max, dtype=np.float32)[None, :, None, None]
+    k = f32_to_bf16_bits(bf16_bits_to_f32(inp["k"]) * 0 + inp["q_f32"][:, :1, None, :] * ramp * 3)
+    kf = bf16_bits_to_f32(k)
+    for path, ctas in (("tcgen05", 0), ("tcgen05", 1), ("simt", 0)):
+        o = binding.decode(dev(inp["q"], "bf16"), dev(k, "bf16"), dev(inp["v"], "bf16"),
+                           torch.from_numpy(inp["lens"]).cuda(), wl.scale, path=path, num_ctas=ctas)
+        ref, _ = oracle_decode(inp["q_f32"], kf, inp["v_f32"], inp["lens"], 1, wl.scale)
+        assert_close(host64(o), ref, "bf16", f"ramp {path} ctas={ctas}")
 
 
 @pytest.mark.parametrize("tile_edge", [1, 63, 64, 65, 127, 128, 129, 255, 256, 257])
