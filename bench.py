@@ -260,7 +260,8 @@ def run_ours(args):
     b, h, g, d = wl.b, wl.h, wl.g, wl.d_k
     path = resolve_path(binding, torch, args.path)
     cache_bytes = wl.b * wl.m_max * wl.g * (wl.d_k + wl.d_v) * wl.elem_bytes
-    copies = max(1, min(8, -(-3 * L2_BYTES // cache_bytes)))      # >= 3x L2 between reuses of one copy
+    # enough copies that >= 2 other steps (and >= 3x L2 of cache) pass between two uses of one copy
+    copies = max(3, min(8, -(-3 * L2_BYTES // cache_bytes) + 1))
     inp = device_inputs(wl, seed=SEED + rank, device="cuda", copies=copies)
     lens_np = inp["lens"]
     lens = torch.from_numpy(lens_np).cuda()

@@ -16,49 +16,60 @@ namespace {
 
 constexpr int kMergeThreads = 128;
 
+// One CTA per (segment, group of heads); each thread merges four consecutive
+// output columns of one head, so the few partial loads of every output are
+// issued by many threads at once instead of walked serially.
 template <typename T>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a, int heads_per_cta) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int64_t s = blockIdx.x;
-  const int seq = int(s / a.g), head = int(s - int64_t(seq) * a.g);
   const int hq = a.hq, D = a.d;
-  T* O = static_cast<T*>(a.o) + (int64_t(seq) * a.h + int64_t(head) * hq) * D;
+  const int chunks = (hq + heads_per_cta - 1) / heads_per_cta;
+  const int64_t s = blockIdx.x / chunks;
+  const int hc = int(blockIdx.x - s * chunks);
+  const int tph = D / 4;                                    // threads per head
+  const int i = hc * heads_per_cta + int(threadIdx.x) / tph;
+  const int c4 = (int(threadIdx.x) % tph) * 4;
+  if (threadIdx.x >= heads_per_cta * tph || i >= hq) return;
+  const int seq = int(s / a.g), head = int(s - int64_t(seq) * a.g);
+  T* O = static_cast<T*>(a.o) + (int64_t(seq) * a.h + int64_t(head) * hq + i) * D + c4;
   const int len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
   if (len == 0) {
-    for (int f = threadIdx.x; f < hq * D; f += kMergeThreads) O[f] = from_f32<T>(0.f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) O[k] = from_f32<T>(0.f);
     return;
   }
   const int2 info = a.ws.seg_info[s];
   if (info.x == info.y) return;
-  for (int f = threadIdx.x; f < hq * D; f += kMergeThreads) {
-    const int i = f / D;
-    float m = -INFINITY, wsum = 0.f, acc = 0.f;
-    for (int k = info.x; k <= info.y; ++k) {
-      const int64_t slot = partial_slot(k, s);
-      const float lse = a.ws.part_lse[slot * hq + i];
-      const float v = a.ws.part_o[slot * hq * D + f];
-      if (lse > m) {
-        const float c = exp2f(m - lse);
-        acc = acc * c + v;
-        wsum = wsum * c + 1.f;
-        m = lse;
-      } else {
-        const float w = exp2f(lse - m);
-        acc = fmaf(w, v, acc);
-        wsum += w;
-      }
-    }
-    O[f] = from_f32<T>(acc / wsum);
+  float m = -INFINITY, wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = info.x; k <= info.y; ++k) {
+    const int64_t slot = partial_slot(k, s);
+    const float lse = a.ws.part_lse[slot * hq + i];
+    const float4 v = *reinterpret_cast<const float4*>(a.ws.part_o + (slot * hq + i) * D + c4);
+    const float mn = fmaxf(m, lse);
+    const float cold = exp2f(m - mn), cnew = exp2f(lse - mn);
+    acc.x = acc.x * cold + cnew * v.x;
+    acc.y = acc.y * cold + cnew * v.y;
+    acc.z = acc.z * cold + cnew * v.z;
+    acc.w = acc.w * cold + cnew * v.w;
+    wsum = wsum * cold + cnew;
+    m = mn;
   }
+  const float inv = 1.f / wsum;
+  O[0] = from_f32<T>(acc.x * inv);
+  O[1] = from_f32<T>(acc.y * inv);
+  O[2] = from_f32<T>(acc.z * inv);
+  O[3] = from_f32<T>(acc.w * inv);
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream) {
-  const int64_t segs = int64_t(a.b) * a.g;
-  if (segs > 0x7fffffff) return cudaErrorInvalidValue;
+  const int heads_per_cta = kMergeThreads / (a.d / 4);
+  const int64_t ctas = int64_t(a.b) * a.g * ((a.hq + heads_per_cta - 1) / heads_per_cta);
+  if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(segs));
+  cfg.gridDim = dim3(unsigned(ctas));
   cfg.blockDim = dim3(kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -67,8 +78,8 @@ cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (dtype == MQA_BF16) return cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16>, a);
-  return cudaLaunchKernelEx(&cfg, merge_kernel<float>, a);
+  if (dtype == MQA_BF16) return cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16>, a, heads_per_cta);
+  return cudaLaunchKernelEx(&cfg, merge_kernel<float>, a, heads_per_cta);
 }
 
 }  // namespace mqa
