@@ -267,7 +267,7 @@ def run_ours(args):
     lens = torch.from_numpy(lens_np).cuda()
     pos = torch.from_numpy(lens_np - 1).cuda()
     out = torch.empty((b, h, wl.d_v), dtype=inp["q"].dtype, device="cuda")
-    ws = torch.empty(binding.decode_workspace_size(b, h, g, wl.d_v), dtype=torch.uint8, device="cuda")
+    ws = binding.new_workspace(b, h, g, wl.d_v)
     stream = torch.cuda.current_stream()
     # one pre-marshalled append and decode per cache copy: each step is two C calls
     appends = [binding.AppendPlan(inp["k"][c], inp["v"][c], inp["k_new"], inp["v_new"], pos) for c in range(copies)]

@@ -83,6 +83,13 @@ def decode_workspace_size(b: int, h: int, g: int, d_v: int) -> int:
     return int(lib().mqa_decode_workspace_size(b, h, g, d_v))
 
 
+def new_workspace(b: int, h: int, g: int, d_v: int, device="cuda"):
+    """A decode workspace (torch uint8 tensor) for these sizes; its contents
+    on entry to a decode do not matter."""
+    import torch
+    return torch.empty(max(256, decode_workspace_size(b, h, g, d_v)), dtype=torch.uint8, device=device)
+
+
 def _dtype_code(t) -> int:
     import torch
     if t.dtype == torch.float32:
@@ -162,7 +169,7 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
     if workspace is None:
         ws = _ws.tensor
         if ws is None or ws.numel() < need or ws.device != q.device:
-            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+            ws = new_workspace(b, h, g, d_v, device=q.device)
             _ws.tensor = ws
         workspace = ws
     opts = DecodeOptions(PATHS[path], int(num_ctas))
@@ -210,8 +217,7 @@ class DecodePlan:
         if out is None:
             out = torch.empty((b, h, d_v), dtype=q.dtype, device=q.device)
         if workspace is None:
-            workspace = torch.empty(max(256, decode_workspace_size(b, h, g, d_v)), dtype=torch.uint8,
-                                    device=q.device)
+            workspace = new_workspace(b, h, g, d_v, device=q.device)
         self.out = out
         self._opts = DecodeOptions(PATHS[path], int(num_ctas))
         self._keep = (q, k_cache, v_cache, lens, out, workspace, status_flags)

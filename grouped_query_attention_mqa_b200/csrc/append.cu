@@ -22,11 +22,13 @@ append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, const ui
   // programmatic dependent launch the wait below orders this kernel's writes
   // after it.  Without PDL it returns at once.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The decode that usually follows may start its set-up now; it waits for
+  // this grid's writes before it reads the cache.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int b = blockIdx.x;
   const int p = __ldg(pos + b);
   if (p < 0 || p >= m_max) {
     if (threadIdx.x == 0) set_flag(flags, MQA_FLAG_POS_SKIPPED);
-    asm volatile("griddepcontrol.launch_dependents;");
     return;
   }
   const int64_t dst_k = (int64_t(b) * m_max + p) * row_k16;
@@ -35,7 +37,6 @@ append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, const ui
     k_cache[dst_k + i] = __ldg(k_new + int64_t(b) * row_k16 + i);
   for (int i = threadIdx.x; i < row_v16; i += kAppendThreads)
     v_cache[dst_v + i] = __ldg(v_new + int64_t(b) * row_v16 + i);
-  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 }  // namespace

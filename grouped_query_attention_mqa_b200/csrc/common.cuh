@@ -115,59 +115,51 @@ __device__ __forceinline__ int cta_of_tile(int64_t t, int64_t total, int active)
   return int(((t + 1) * int64_t(active) - 1) / total);
 }
 
-template <int NT>
-__device__ __forceinline__ int64_t block_sum_i64(int64_t v, int64_t* red) {
-  static_assert(NT % 32 == 0, "whole warps");
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  __syncthreads();
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  int64_t s = 0;
-#pragma unroll
-  for (int i = 0; i < NT / 32; ++i) s += red[i];
-  return s;
-}
-
 // Every CTA derives the same partition from lens.  Thread i sums the tiles of
-// a contiguous block of sequences, a block-wide sum gives T, an exclusive scan
-// of the per-thread sums locates this CTA's first tile, and the thread holding
-// it walks its block to find the sequence.  Cost: O(b / NT) loads per thread.
-// `red` needs NT/32 + NT + 2 int64 of shared memory.
+// a contiguous block of sequences; a warp shuffle scan plus a scan of the warp
+// totals gives T and this thread's exclusive prefix; the thread whose block
+// holds this CTA's first tile walks its block to find the sequence.
+// Cost: O(b / NT) loads per thread and three block barriers.
+// `red` needs NT/32 + 2 int64 of shared memory.
 template <int NT>
 __device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile,
                                int grid, int cta, int32_t* flags, int64_t* red) {
+  static_assert(NT % 32 == 0, "whole warps");
   const int per = (b + NT - 1) / NT;
   const int s0 = min(b, int(threadIdx.x) * per);
   const int s1 = min(b, s0 + per);
   int64_t mine = 0;
   for (int s = s0; s < s1; ++s)
     mine += int64_t(g) * tiles_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), tile);
-  int64_t* warp_red = red;
-  int64_t* incl = red + NT / 32;
-  int64_t* out = incl + NT;
-  const int64_t total = block_sum_i64<NT>(mine, warp_red);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  int64_t* wtot = red;
+  int64_t* out = red + NT / 32;
+  __syncthreads();
+  if (lane == 31) wtot[warp] = x;
+  __syncthreads();
+  int64_t total = 0, before = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const int64_t v = wtot[w];
+    total += v;
+    if (w < warp) before += v;
+  }
+  const int64_t excl = before + x - mine;
   Sched sc;
   sc.total = total;
   sc.active = int(total < grid ? total : int64_t(grid));
   sc.t_begin = sc.t_end = 0;
   sc.seq = 0;
   sc.seq_base = 0;
-  if (cta >= sc.active) return sc;
+  if (cta >= sc.active) return sc;   // uniform across the CTA
   sc.t_begin = range_start(cta, total, sc.active);
   sc.t_end = range_start(int64_t(cta) + 1, total, sc.active);
-  // inclusive scan of per-thread tile sums (NT is small: a plain two-pass scan
-  // through shared memory is enough)
-  incl[threadIdx.x] = mine;
-  __syncthreads();
-  for (int off = 1; off < NT; off <<= 1) {
-    int64_t add = threadIdx.x >= off ? incl[threadIdx.x - off] : 0;
-    __syncthreads();
-    incl[threadIdx.x] += add;
-    __syncthreads();
-  }
-  const int64_t excl = incl[threadIdx.x] - mine;
   if (sc.t_begin >= excl && sc.t_begin < excl + mine) {
     int64_t base = excl;
     for (int s = s0; s < s1; ++s) {
@@ -184,6 +176,122 @@ __device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, i
   sc.seq = int(out[0]);
   sc.seq_base = out[1];
   return sc;
+}
+
+// Weighted partition (tensor-core path).  Positions are counted in units of a
+// quarter tile, and every segment starts with `xw` extra units that stand for
+// the fixed cost a CTA pays to enter a segment (its queries, a full max
+// reduction, writing the output).  Segment s of sequence b spans
+// xw + 4*nb units; tile k of it starts xw + 4*k units after the segment does.
+// CTA c owns the tiles whose start unit lies in [c*W/A, (c+1)*W/A), so a CTA
+// whose range crosses segment starts gets correspondingly fewer tiles.  With
+// A <= W / (xw + 4) every range holds at least one tile start.
+struct WSched {
+  Sched s;
+  int64_t wtotal;     // W: units over all segments
+  int64_t seq_ubase;  // first unit of sequence s.seq
+};
+
+__device__ __forceinline__ int64_t seq_units(int nb, int g, int xw) {
+  return nb > 0 ? int64_t(g) * (xw + 4 * int64_t(nb)) : 0;
+}
+
+// CTA whose unit range holds unit u.
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t wtotal, int active) {
+  return int(((u + 1) * int64_t(active) - 1) / wtotal);
+}
+
+template <int NT>
+__device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile,
+                                         int grid, int cta, int32_t* flags, int64_t* red, int xw) {
+  static_assert(NT % 32 == 0, "whole warps");
+  const int per = (b + NT - 1) / NT;
+  const int s0 = min(b, int(threadIdx.x) * per);
+  const int s1 = min(b, s0 + per);
+  int64_t my_t = 0, my_u = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int nb = tiles_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), tile);
+    my_t += int64_t(g) * nb;
+    my_u += seq_units(nb, g, xw);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t xt = my_t, xu = my_u;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t yt = __shfl_up_sync(0xffffffffu, xt, o);
+    const int64_t yu = __shfl_up_sync(0xffffffffu, xu, o);
+    if (lane >= o) {
+      xt += yt;
+      xu += yu;
+    }
+  }
+  int64_t* wt = red;                 // [NT/32] warp tile totals
+  int64_t* wu = red + NT / 32;       // [NT/32] warp unit totals
+  int64_t* out = red + 2 * (NT / 32);
+  __syncthreads();
+  if (lane == 31) {
+    wt[warp] = xt;
+    wu[warp] = xu;
+  }
+  __syncthreads();
+  int64_t T = 0, W = 0, bt = 0, bu = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const int64_t vt = wt[w], vu = wu[w];
+    T += vt;
+    W += vu;
+    if (w < warp) {
+      bt += vt;
+      bu += vu;
+    }
+  }
+  const int64_t excl_t = bt + xt - my_t, excl_u = bu + xu - my_u;
+  WSched ws;
+  ws.s.total = T;
+  ws.wtotal = W;
+  const int64_t cap = W / (xw + 4);
+  ws.s.active = int(cap < grid ? cap : int64_t(grid));
+  ws.s.t_begin = ws.s.t_end = 0;
+  ws.s.seq = 0;
+  ws.s.seq_base = 0;
+  ws.seq_ubase = 0;
+  if (cta >= ws.s.active) return ws;   // uniform across the CTA
+  const int64_t u0 = (int64_t(cta) * W) / ws.s.active;
+  const int64_t u1 = ((int64_t(cta) + 1) * W) / ws.s.active;
+  // Tiles whose start unit is below u (< W), computed by the thread whose
+  // block of sequences holds u; also the sequence holding u and its bases.
+  auto locate = [&](int64_t u, int64_t* dst, bool with_seq) {
+    if (!(u >= excl_u && u < excl_u + my_u)) return;
+    int64_t tb = excl_t, ub = excl_u;
+    for (int s = s0; s < s1; ++s) {
+      const int nb = tiles_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), tile);
+      const int64_t su = seq_units(nb, g, xw);
+      if (u < ub + su) {
+        const int64_t seglen = xw + 4 * int64_t(nb);
+        const int64_t rel = u - ub;
+        const int64_t j = rel / seglen, off = rel - j * seglen;
+        const int64_t cnt = off <= xw ? 0 : (off - xw + 3) / 4;
+        dst[0] = tb + j * nb + cnt;
+        if (with_seq) {
+          dst[1] = s;
+          dst[2] = tb;
+          dst[3] = ub;
+        }
+        return;
+      }
+      tb += int64_t(g) * nb;
+      ub += su;
+    }
+  };
+  locate(u0, out, true);
+  if (u1 < W) locate(u1, out + 4, false);
+  __syncthreads();
+  ws.s.t_begin = out[0];
+  ws.s.seq = int(out[1]);
+  ws.s.seq_base = out[2];
+  ws.seq_ubase = out[3];
+  ws.s.t_end = u1 == W ? T : out[4];
+  return ws;
 }
 
 // Walks the tile numbering forward from a known sequence.

@@ -48,12 +48,13 @@ using namespace sm100;
 
 constexpr int kTile = 128;                   // cache rows per tile (the MMA M)
 constexpr int kD = 128;                      // head size
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;             // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr int kNpv = 64;                     // N of the P.V product (P padded with zero columns)
 constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte swizzle column
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
+constexpr int kSegUnits = 6;                 // cost of entering a segment, in quarter tiles (partition weight)
 constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O double buffer at [128, 256)
 constexpr uint32_t kOCol = 128;
 constexpr uint32_t kMaxDynSmem = 232448;     // 227 KB opt-in limit per CTA
@@ -78,16 +79,18 @@ struct TcCfg {
   static constexpr uint32_t kRed = (kAbort + 4 + 15) / 16 * 16;  // [4][NP] f32
   static constexpr uint32_t kMref = kRed + 4 * NP * 4;
   static constexpr uint32_t kAlpha = kMref + NP * 4;
-  static constexpr uint32_t kLsum = kAlpha + NP * 4;
-  static constexpr uint32_t kEnd = kLsum + NP * 4;
+  static constexpr uint32_t kRedL = kAlpha + NP * 4;             // [4][NP] f32: per-warp head sums
+  static constexpr uint32_t kLinv = kRedL + 4 * NP * 4;          // [2][NP]: 1 / l per segment parity
+  static constexpr uint32_t kLse = kLinv + 2 * NP * 4;           // [2][NP]: log2-sum-exp per segment parity
+  static constexpr uint32_t kEnd = kLse + 2 * NP * 4;
   static constexpr uint32_t kAlloc = kEnd + 1024;             // room to align the base to 1024 bytes
   static constexpr uint32_t kSched = kP;                      // start-up scratch, before P is zeroed
   static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kQBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kAlloc <= kMaxDynSmem, "shared memory budget");
-  static_assert((kThreads / 32 + kThreads + 2) * 8 <= kPBytes, "schedule scratch fits in P");
+  static_assert((2 * (kThreads / 32) + 8) * 8 <= kPBytes, "schedule scratch fits in P");
 };
 
-__device__ __forceinline__ void named_barrier_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_barrier_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Barriers of the four softmax warps that also reduce a per-thread flag, so
 // that every thread takes the same branch afterwards (a thread that gave up a
@@ -97,7 +100,7 @@ __device__ __forceinline__ bool softmax_barrier_and(bool v) {
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "bar.red.and.pred po, 1, 256, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
       : "r"(uint32_t(v))
@@ -109,7 +112,7 @@ __device__ __forceinline__ bool softmax_barrier_or(bool v) {
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.or.pred po, 1, 128, pi;\n\t"
+      "bar.red.or.pred po, 1, 256, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
       : "r"(uint32_t(v))
@@ -158,23 +161,32 @@ __device__ __forceinline__ bool wait_bar(const Roles& r, uint32_t bar, uint32_t 
 
 // Walks the CTA's tiles in order and tells each role what a tile is.  Only
 // the first step divides; later steps count (tile, head, sequence) forward.
+// It also tracks the partition units, so that the owner of any tile can be
+// computed.
 struct TileWalk {
   int64_t t;                 // current tile number
   int64_t base;              // first tile of the current sequence
+  int64_t ubase;             // first partition unit of the current sequence
   int seq, head, k, nb, len;
   int sidx;                  // segment number within this CTA
   TileCoord tc;
   bool first, last;
-  __device__ TileWalk(const DecodeArgs& a, const Sched& sc) : t(sc.t_begin - 1), sidx(-1) {
-    Cursor cu = cursor_at(a.lens, a.m_max, kTile, sc.seq, sc.seq_base);
-    cursor_seek(cu, a.lens, a.g, a.m_max, kTile, sc.t_begin);
-    seq = cu.seq;
-    base = cu.base;
-    nb = cu.nb;
-    len = cu.len;
-    const int64_t rel = sc.t_begin - cu.base;
-    head = int(rel / cu.nb);
-    k = int(rel - int64_t(head) * cu.nb) - 1;   // next() advances to the first tile
+  __device__ TileWalk(const DecodeArgs& a, const WSched& ws) : t(ws.s.t_begin - 1), sidx(-1) {
+    seq = ws.s.seq;
+    base = ws.s.seq_base;
+    ubase = ws.seq_ubase;
+    len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
+    nb = tiles_of(len, kTile);
+    while (ws.s.t_begin >= base + int64_t(a.g) * nb) {   // the first tile may lie in a later sequence
+      base += int64_t(a.g) * nb;
+      ubase += seq_units(nb, a.g, kSegUnits);
+      ++seq;
+      len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
+      nb = tiles_of(len, kTile);
+    }
+    const int64_t rel = ws.s.t_begin - base;
+    head = int(rel / nb);
+    k = int(rel - int64_t(head) * nb) - 1;   // next() advances to the first tile
   }
   __device__ void next(const DecodeArgs& a, const Sched& sc) {
     ++t;
@@ -183,6 +195,7 @@ struct TileWalk {
       if (++head == a.g) {
         head = 0;
         base += int64_t(a.g) * nb;
+        ubase += seq_units(nb, a.g, kSegUnits);
         do {
           ++seq;
           len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
@@ -202,20 +215,25 @@ struct TileWalk {
     last = (k == nb - 1) || (t + 1 == sc.t_end);
     if (first) ++sidx;
   }
+  // partition unit where the current segment's last tile starts
+  __device__ int64_t seg_last_unit() const {
+    return ubase + int64_t(head) * (kSegUnits + 4 * int64_t(nb)) + kSegUnits + 4 * int64_t(nb - 1);
+  }
 };
 
 // K ring and the per-segment Q (kIsK), or the V ring.
 template <int NP, int SK, int SV, bool kIsK>
-__device__ void producer(const DecodeArgs& a, const Sched& sc, const Roles& r, const CUtensorMap* tm_kv,
+__device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, const CUtensorMap* tm_kv,
                          const CUtensorMap* tm_q) {
   using C = TcCfg<NP, SK, SV>;
+  const Sched& sc = ws.s;
   constexpr int S = kIsK ? SK : SV;
   constexpr int kFull = kIsK ? C::kKFull : C::kVFull;
   constexpr int kEmpty = kIsK ? C::kKEmpty : C::kVEmpty;
   constexpr uint32_t kRing = kIsK ? C::kK : C::kV;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  TileWalk w(a, sc);
+  TileWalk w(a, ws);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t i = 0;
   int q_issued = -1;
@@ -248,64 +266,96 @@ __device__ void producer(const DecodeArgs& a, const Sched& sc, const Roles& r, c
       mbar_wait(bar(C::kQFull + (sq & 1)), uint32_t(sq >> 1) & 1, kTimeoutNs);
 }
 
+// One thread issues every tensor-core product.  S(j) = K Q^T may run once
+// K(j) has landed (and, for a segment's first tile, its Q) and S buffer j&1 is
+// free, i.e. P(j-2) has been consumed; O += V^T P(j) once P(j) is written and
+// V(j) has landed.  The two streams are independent, so the thread polls both
+// and issues whichever is ready: a late K tile never holds up a P.V product
+// the softmax warps are waiting for.
 template <int NP, int SK, int SV>
-__device__ void mma_issuer(const DecodeArgs& a, const Sched& sc, const Roles& r) {
+__device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
   using C = TcCfg<NP, SK, SV>;
+  const Sched& sc = ws.s;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int64_t n = sc.t_end - sc.t_begin;
-  TileWalk wq(a, sc), wp(a, sc);   // look-ahead walker for S, trailing walker for O
+  TileWalk wq(a, ws), wp(a, ws);   // walkers for the S stream and the O stream
+  const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);           // K-major, rows of 128 B
+  const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
+  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
+  const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);   // MN-major P
 
-  auto issue_qk = [&](int64_t i) -> bool {
-    wq.next(a, sc);
-    const int st = int(i % SK);
-    const int qb = wq.sidx & 1;
-    if (wq.first && !wait_bar(r, bar(C::kQFull + qb), uint32_t(wq.sidx >> 1) & 1)) return false;
-    if (!wait_bar(r, bar(C::kKFull + st), uint32_t(i / SK) & 1)) return false;
-    tc_fence_after();
-    const uint32_t kbase = r.sbase + C::kK + st * kTileBytes;
-    const uint32_t qbase = r.sbase + C::kQ + qb * C::kQBytes;
-    const uint32_t d = r.tmem + uint32_t(i & 1) * NP;
+  int64_t iq = 0, ip = 0;          // next S and next O product
+  bool q_walked = false, p_walked = false;
+  uint64_t idle_since = 0;
+  uint32_t idle_polls = 0;
+  while (ip < n) {
+    bool progressed = false;
+    // S(iq): needs K(iq), Q of its segment, and P(iq-2) consumed (iq <= ip + 1)
+    if (iq < n && iq <= ip + 1) {
+      if (!q_walked) {
+        wq.next(a, sc);
+        q_walked = true;
+      }
+      const int st = int(iq % SK);
+      const int qb = wq.sidx & 1;
+      if ((!wq.first || mbar_test(bar(C::kQFull + qb), uint32_t(wq.sidx >> 1) & 1)) &&
+          mbar_test(bar(C::kKFull + st), uint32_t(iq / SK) & 1)) {
+        tc_fence_after();
+        // descriptors differ only in their start address (bits 0-13, 16-byte units)
+        const uint64_t ka = kdesc0 + ((st * kTileBytes) >> 4);
+        const uint64_t qa = qdesc0 + ((qb * C::kQBytes) >> 4);
+        const uint32_t d = r.tmem + uint32_t(iq & 1) * NP;
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-      const uint32_t qoff = (kk >> 2) * (NP * 128) + (kk & 3) * 32;
-      mma_bf16_ss(d, smem_desc_sw128(kbase + koff, 16, 1024), smem_desc_sw128(qbase + qoff, 16, 1024), idesc_qk,
-                  kk > 0);
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
+        }
+        mma_commit(bar(C::kSFull + (iq & 1)));
+        mma_commit(bar(C::kKEmpty + st));
+        if (wq.last) mma_commit(bar(C::kQEmpty + qb));
+        ++iq;
+        q_walked = false;
+        progressed = true;
+      }
     }
-    mma_commit(bar(C::kSFull + (i & 1)));
-    mma_commit(bar(C::kKEmpty + st));
-    if (wq.last) mma_commit(bar(C::kQEmpty + qb));
-    return true;
-  };
-  auto issue_pv = [&](int64_t i) -> bool {
-    wp.next(a, sc);
-    const int st = int(i % SV);
-    const int ob = wp.sidx & 1;
-    if (!wait_bar(r, bar(C::kPFull), uint32_t(i & 1))) return false;
-    if (!wait_bar(r, bar(C::kVFull + st), uint32_t(i / SV) & 1)) return false;
-    if (wp.first && wp.sidx >= 2 && !wait_bar(r, bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))
-      return false;
-    tc_fence_after();
-    const uint32_t vbase = r.sbase + C::kV + st * kTileBytes;
-    const uint32_t pbase = r.sbase + C::kP;
-    const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
+    // O += V^T P(ip): needs P(ip), V(ip) and, for a segment's first tile, its O buffer
+    if (ip < iq) {
+      if (!p_walked) {
+        wp.next(a, sc);
+        p_walked = true;
+      }
+      const int st = int(ip % SV);
+      const int ob = wp.sidx & 1;
+      if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) && mbar_test(bar(C::kVFull + st), uint32_t(ip / SV) & 1) &&
+          (!wp.first || wp.sidx < 2 || mbar_test(bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))) {
+        tc_fence_after();
+        const uint64_t va = vdesc0 + ((st * kTileBytes) >> 4);
+        const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
+        const uint32_t acc0 = wp.first ? 0u : 1u;
 #pragma unroll
-    for (int kk = 0; kk < kTile / 16; ++kk) {
-      mma_bf16_ss(d, smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024),
-                  smem_desc_sw128(pbase + kk * 2048, kHalfBytes, 1024), idesc_pv, (kk > 0 || !wp.first) ? 1u : 0u);
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        mma_commit(bar(C::kOFull));
+        mma_commit(bar(C::kVEmpty + st));
+        ++ip;
+        p_walked = false;
+        progressed = true;
+      }
     }
-    mma_commit(bar(C::kOFull));
-    mma_commit(bar(C::kVEmpty + st));
-    return true;
-  };
-
-  if (n > 0 && issue_qk(0)) {
-    for (int64_t i = 0; i < n; ++i) {
-      if (*r.abort) break;
-      if (i + 1 < n && !issue_qk(i + 1)) break;
-      if (!issue_pv(i)) break;
+    if (progressed) {
+      idle_polls = 0;
+    } else if ((++idle_polls & 1023u) == 0) {   // bounded: give up after the timeout without progress
+      const uint64_t now = globaltimer_ns();
+      if (idle_polls == 1024) {
+        idle_since = now;
+      } else if (now - idle_since > kTimeoutNs || *r.abort) {
+        *r.abort = 1;
+        set_flag(r.flags, MQA_FLAG_PIPE_TIMEOUT);
+        break;
+      }
     }
   }
   // every MMA issued above has completed before tensor memory is released
@@ -314,78 +364,143 @@ __device__ void mma_issuer(const DecodeArgs& a, const Sched& sc, const Roles& r)
 }
 
 template <int NP, int SK, int SV>
-__device__ void softmax_epilogue(const DecodeArgs& a, const Sched& sc, const Roles& r, int warp, int lane) {
+__device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Roles& r, int warp, int lane) {
   using C = TcCfg<NP, SK, SV>;
+  const Sched& sc = ws.s;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   auto wait = [&](int id, uint32_t parity) { return mbar_wait(bar(id), parity, kTimeoutNs); };
-  constexpr int NCH = NP / 16;
+  constexpr int CPT = NP / 2;                      // heads per thread: two warps share each row
+  constexpr int W = CPT < 16 ? CPT : 16;           // transpose-reduction width
   const int q4 = warp & 3;                         // TMEM lane quarter this warp may access
-  const int sw = warp - 2;                         // index within the softmax group
+  const int grp = (warp - 2) >> 2;                 // column group: heads [grp*CPT, grp*CPT + CPT)
+  const int gw = (warp - 2) & 3;                   // warp index within the column group
+  const int col0 = grp * CPT;
+  const int tid = threadIdx.x - 64;                // 0..255 over the softmax warps
   const int row = 32 * q4 + lane;                  // cache row of the tile (S), output column (O)
   const uint32_t t_lane = r.tmem + (uint32_t(32 * q4) << 16);
-  float* red = reinterpret_cast<float*>(r.smem + C::kRed);
+  float* red = reinterpret_cast<float*>(r.smem + C::kRed);      // [4][NP]
   float* mref = reinterpret_cast<float*>(r.smem + C::kMref);
   float* alpha = reinterpret_cast<float*>(r.smem + C::kAlpha);
-  float* lsum = reinterpret_cast<float*>(r.smem + C::kLsum);
+  float* redl = reinterpret_cast<float*>(r.smem + C::kRedL);    // [4][NP]
+  float* linv = reinterpret_cast<float*>(r.smem + C::kLinv);
+  float* lse2 = reinterpret_cast<float*>(r.smem + C::kLse);
   const float c = a.scale * kLog2e;
   const int hq = a.hq;
-  float lpart[NP];
-  float sv[NP];
-  // reference max per head (log2 units): mirrored in registers when they suffice
-  constexpr bool kMrRegs = NP <= 32;
-  float mr[kMrRegs ? NP : 1];
-  auto mref_of = [&](int k) -> float {
-    if constexpr (kMrRegs) return mr[k];
-    else return mref[k];
-  };
-  TileWalk w(a, sc);
+  float lpart[CPT];                                // this row's share of the per-head sums
+  float sv[CPT];                                   // this row's scaled logits (log2 units)
+  float mr[CPT];                                   // reference max per head, mirrored from smem
+  TileWalk w(a, ws);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t pv_waited = -1;
   bool failed = false;
+
+  // A finished segment whose output is written one tile later, once the P.V
+  // product of its last tile is known to have completed.
+  struct Pending {
+    bool on;
+    int sidx, seq, head;
+    int64_t seg;
+    bool whole, owns_first;
+    int64_t seg_last_unit;   // partition unit where the segment's last tile starts
+  } pend;
+  pend.on = false;
+
+  // Write a finished segment: O^T from tensor memory times 1/l, staged through
+  // the (idle) P buffer as [head][column] and stored with 16-byte copies; then
+  // the pad columns of P are zeroed again and the O buffer is released.
+  auto epilogue = [&](const Pending& e) {
+    const int pb = e.sidx & 1;
+    unsigned char* stage = r.smem + C::kP;
+    constexpr int kPass = 32;                          // heads per fp32 pass (16 KB)
+    const int passes = e.whole ? 1 : (hq + kPass - 1) / kPass;
+    const int64_t slot = partial_slot(blockIdx.x, e.seg);
+    float v[CPT], li[CPT];
+    tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) li[k] = linv[pb * NP + col0 + k];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) v[k] *= li[k];
+    for (int ps = 0; ps < passes; ++ps) {
+      const int c0 = e.whole ? 0 : ps * kPass;
+      const int nc = e.whole ? hq : min(kPass, hq - c0);
+      if (e.whole) {
+        __nv_bfloat16* st16 = reinterpret_cast<__nv_bfloat16*>(stage) + row;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+          if (col0 + k < hq) st16[(col0 + k) * kD] = __float2bfloat16_rn(v[k]);
+      } else {
+        float* st32 = reinterpret_cast<float*>(stage) + row;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+          const int col = col0 + k - c0;
+          if (col >= 0 && col < nc) st32[col * kD] = v[k];
+        }
+      }
+      named_barrier_softmax();
+      const int esz = e.whole ? 2 : 4;
+      const int chunks = nc * kD * esz / 16;
+      uint4* dst = e.whole ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
+                                                      (int64_t(e.seq) * a.h + int64_t(e.head) * hq) * kD)
+                           : reinterpret_cast<uint4*>(a.ws.part_o + (slot * hq + c0) * kD);
+      const uint4* src = reinterpret_cast<const uint4*>(stage);
+      for (int k = tid; k < chunks; k += 256) dst[k] = src[k];
+      named_barrier_softmax();
+    }
+    if (warp == 2) {
+      if (!e.whole)
+        for (int col = lane; col < hq; col += 32) a.ws.part_lse[slot * hq + col] = lse2[pb * NP + col];
+      if (e.owns_first && lane == 0)
+        a.ws.seg_info[e.seg] = make_int2(blockIdx.x, cta_of_unit(e.seg_last_unit, ws.wtotal, sc.active));
+    }
+    if constexpr (NP < 64) {   // the staging overwrote the zero pad columns of P
+      if (grp == 1) {
+        unsigned char* prow0 = r.smem + C::kP + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+        for (int c8 = NP / 8; c8 < 8; ++c8)
+          *reinterpret_cast<uint4*>(prow0 + ((c8 ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(bar(C::kOFree + pb));
+  };
+
   for (int64_t i = 0; i < n; ++i) {
     w.next(a, sc);
     if (w.first) {
 #pragma unroll
-      for (int k = 0; k < NP; ++k) lpart[k] = 0.f;
+      for (int k = 0; k < CPT; ++k) lpart[k] = 0.f;
     }
     bool ok = wait(C::kSFull + (i & 1), uint32_t(i >> 1) & 1);
     tc_fence_after();
     const bool valid = row < w.tc.rows;
-    // scaled logits (log2 units) of this thread's row
+    tmem_ld<CPT>(t_lane + uint32_t(i & 1) * NP + col0, sv);
 #pragma unroll
-    for (int ch = 0; ch < NP / 32; ++ch) {
-      float v[32];
-      tmem_ld32(t_lane + uint32_t(i & 1) * NP + ch * 32, v);
-#pragma unroll
-      for (int k = 0; k < 32; ++k) sv[ch * 32 + k] = v[k];
-    }
-    if constexpr (NP % 32 != 0) {
-      float v[16];
-      tmem_ld16(t_lane + uint32_t(i & 1) * NP + (NP / 32) * 32, v);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) sv[(NP / 32) * 32 + k] = v[k];
-    }
-#pragma unroll
-    for (int k = 0; k < NP; ++k) sv[k] = valid ? sv[k] * c : -INFINITY;
+    for (int k = 0; k < CPT; ++k) sv[k] = valid ? sv[k] * c : -INFINITY;
     // Does any logit of a real head exceed the reference max by the threshold?
     bool exceed = false;
     if (!w.first) {
+      float d[CPT];
 #pragma unroll
-      for (int k = 0; k < NP; ++k) exceed |= (k < hq) && (sv[k] > mref_of(k) + kRescaleThreshold);
+      for (int k = 0; k < CPT; ++k) d[k] = (col0 + k < hq) ? sv[k] - mr[k] : -INFINITY;
+#pragma unroll
+      for (int span = CPT / 2; span >= 1; span >>= 1)
+#pragma unroll
+        for (int k = 0; k < span; ++k) d[k] = fmaxf(d[k], d[k + span]);
+      exceed = d[0] > kRescaleThreshold;
     }
     const bool full = w.first || softmax_barrier_or(exceed);
     if (full) {   // column maxima of the tile and the new reference max
 #pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        float v[16];
+      for (int ch = 0; ch < CPT / W; ++ch) {
+        float v[W];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = sv[ch * 16 + k];
-        const float mx = transpose_reduce<16, true>(v, lane);
-        if (lane < 16) red[sw * NP + ch * 16 + lane] = mx;
+        for (int k = 0; k < W; ++k) v[k] = sv[ch * W + k];
+        const float mx = transpose_reduce<W, true>(v, lane);
+        if (lane < W) red[gw * NP + col0 + ch * W + lane] = mx;
       }
       named_barrier_softmax();
-      if (sw == 0) {
-        for (int col = lane; col < NP; col += 32) {
+      if (gw == 0) {   // one warp per column group decides for its heads
+        for (int col = col0 + lane; col < col0 + CPT; col += 32) {
           const float mt = fmaxf(fmaxf(red[col], red[NP + col]), fmaxf(red[2 * NP + col], red[3 * NP + col]));
           float mn = mt, al = 1.f;
           if (!w.first) {
@@ -401,10 +516,8 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const Sched& sc, const Rol
         }
       }
       named_barrier_softmax();
-      if constexpr (kMrRegs) {
 #pragma unroll
-        for (int k = 0; k < NP; ++k) mr[k] = mref[k];
-      }
+      for (int k = 0; k < CPT; ++k) mr[k] = mref[col0 + k];
     }
     // O(i-1) must be complete before O is rescaled and before P(i) overwrites
     // the P buffer it read; a ragged tile needs its V rows landed before the
@@ -418,47 +531,55 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const Sched& sc, const Rol
     if (w.tc.rows < kTile) ok2 = wait(C::kVFull + st, uint32_t(i / SV) & 1) && ok2;
     if (!softmax_barrier_and(ok && ok2)) { failed = true; break; }
     tc_fence_after();
+    if (pend.on) {
+      epilogue(pend);
+      pend.on = false;
+    }
     if (full && !w.first) {
+      float al[CPT];
 #pragma unroll
-      for (int k = 0; k < NP; ++k) lpart[k] *= alpha[k];
-      // rescale the O accumulated so far (thread = output column)
-      const uint32_t oc = t_lane + kOCol + uint32_t(w.sidx & 1) * kNpv;
-#pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        float v[16];
-        tmem_ld16(oc + ch * 16, v);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] *= alpha[ch * 16 + k];
-        tmem_st16(oc + ch * 16, v);
+      for (int k = 0; k < CPT; ++k) {
+        al[k] = alpha[col0 + k];
+        lpart[k] *= al[k];
       }
+      // rescale the O accumulated so far (thread = output column, its heads)
+      const uint32_t oc = t_lane + kOCol + uint32_t(w.sidx & 1) * kNpv + col0;
+      float v[CPT];
+      tmem_ld<CPT>(oc, v);
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) v[k] *= al[k];
+      tmem_st<CPT>(oc, v);
       tmem_wait_st();
     }
     // P = exp2(s - m), bf16, into the MN-major 128-byte-swizzled P buffer
     unsigned char* prow = r.smem + C::kP + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-    for (int c8 = 0; c8 < NP / 8; ++c8) {
+    for (int c8 = 0; c8 < CPT / 8; ++c8) {
       uint32_t packed[4];
 #pragma unroll
       for (int k2 = 0; k2 < 4; ++k2) {
-        const int col = c8 * 8 + k2 * 2;
-        const float p0 = col < hq ? ex2_approx(sv[col] - mref_of(col)) : 0.f;
-        const float p1 = col + 1 < hq ? ex2_approx(sv[col + 1] - mref_of(col + 1)) : 0.f;
-        lpart[col] += p0;
-        lpart[col + 1] += p1;
+        const int k = c8 * 8 + k2 * 2;
+        const float p0 = col0 + k < hq ? ex2_approx(sv[k] - mr[k]) : 0.f;
+        const float p1 = col0 + k + 1 < hq ? ex2_approx(sv[k + 1] - mr[k + 1]) : 0.f;
+        lpart[k] += p0;
+        lpart[k + 1] += p1;
         __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
         packed[k2] = *reinterpret_cast<uint32_t*>(&b2);
       }
-      *reinterpret_cast<uint4*>(prow + ((c8 ^ (row & 7)) << 4)) =
+      const int chunk = col0 / 8 + c8;
+      *reinterpret_cast<uint4*>(prow + ((chunk ^ (row & 7)) << 4)) =
           make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    if (!valid) {
+    if (w.tc.rows < kTile) {
       // rows past the sequence end were loaded too; zero them in V so that
-      // P = 0 times whatever they hold contributes exactly 0
-      unsigned char* v0 = r.smem + C::kV + st * kTileBytes + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
-        *reinterpret_cast<uint4*>(v0 + c16 * 16) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(v0 + kHalfBytes + c16 * 16) = make_uint4(0, 0, 0, 0);
+      // P = 0 times whatever they hold contributes exactly 0.  Consecutive
+      // threads take consecutive 16-byte pieces of a row (no bank conflicts).
+      unsigned char* vst = r.smem + C::kV + st * kTileBytes;
+      const int nchunks = (kTile - w.tc.rows) * 16;
+      for (int k = tid; k < nchunks; k += 256) {
+        const int vr = w.tc.rows + (k >> 4), half = (k >> 3) & 1, c16 = k & 7;
+        *reinterpret_cast<uint4*>(vst + half * kHalfBytes + (vr >> 3) * 1024 + (vr & 7) * 128 + c16 * 16) =
+            make_uint4(0, 0, 0, 0);
       }
     }
     fence_proxy_async_smem();
@@ -466,56 +587,44 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const Sched& sc, const Rol
     mbar_arrive(bar(C::kPFull));
 
     if (w.last) {
-      ok = wait(C::kOFull, uint32_t(i) & 1);
-      pv_waited = i;
-      // per-head sums over the 128 rows
+      // per-head sums over the 128 rows; the output follows one tile later
 #pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        float v[16];
+      for (int ch = 0; ch < CPT / W; ++ch) {
+        float v[W];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = lpart[ch * 16 + k];
-        const float s = transpose_reduce<16, false>(v, lane);
-        if (lane < 16) red[sw * NP + ch * 16 + lane] = s;
+        for (int k = 0; k < W; ++k) v[k] = lpart[ch * W + k];
+        const float sum = transpose_reduce<W, false>(v, lane);
+        if (lane < W) redl[gw * NP + col0 + ch * W + lane] = sum;
       }
-      if (!softmax_barrier_and(ok)) { failed = true; break; }
-      tc_fence_after();
-      if (sw == 0)
-        for (int col = lane; col < NP; col += 32)
-          lsum[col] = red[col] + red[NP + col] + red[2 * NP + col] + red[3 * NP + col];
       named_barrier_softmax();
-      const bool owns_first = w.tc.seg_t0 >= sc.t_begin;
-      const bool whole = owns_first && (w.tc.seg_t0 + w.tc.nb <= sc.t_end);
-      const int64_t slot = partial_slot(blockIdx.x, w.tc.seg);
-      const uint32_t oc = t_lane + kOCol + uint32_t(w.sidx & 1) * kNpv;
-      const int64_t obase = (int64_t(w.tc.seq) * a.h + int64_t(w.tc.head) * hq) * kD;
-#pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        float v[16];
-        tmem_ld16(oc + ch * 16, v);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int col = ch * 16 + k;
-          if (col < hq) {
-            const float val = v[k] / lsum[col];
-            if (whole)
-              static_cast<__nv_bfloat16*>(a.o)[obase + int64_t(col) * kD + row] = __float2bfloat16_rn(val);
-            else
-              a.ws.part_o[(slot * hq + col) * kD + row] = val;
-          }
+      const int pb = w.sidx & 1;
+      if (gw == 0)
+        for (int col = col0 + lane; col < col0 + CPT; col += 32) {
+          const float l = redl[col] + redl[NP + col] + redl[2 * NP + col] + redl[3 * NP + col];
+          linv[pb * NP + col] = rcp_approx(l);
+          lse2[pb * NP + col] = mref[col] + lg2_approx(l);
         }
-      }
-      if (sw == 0) {
-        if (!whole)
-          for (int col = lane; col < hq; col += 32) a.ws.part_lse[slot * hq + col] = mref[col] + log2f(lsum[col]);
-        if (owns_first && lane == 0)
-          a.ws.seg_info[w.tc.seg] =
-              make_int2(blockIdx.x, cta_of_tile(w.tc.seg_t0 + w.tc.nb - 1, sc.total, sc.active));
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::kOFree + (w.sidx & 1)));
+      pend.on = true;
+      pend.sidx = w.sidx;
+      pend.seq = w.tc.seq;
+      pend.head = w.tc.head;
+      pend.seg = w.tc.seg;
+      pend.owns_first = w.tc.seg_t0 >= sc.t_begin;
+      pend.whole = pend.owns_first && (w.tc.seg_t0 + w.tc.nb <= sc.t_end);
+      pend.seg_last_unit = w.seg_last_unit();
     }
   }
-  if (failed && threadIdx.x == 64) {
+  if (!failed && pend.on) {   // the CTA's last segment: wait for its final P.V, then write it
+    bool ok = true;
+    if (pv_waited < n - 1) ok = wait(C::kOFull, uint32_t(n - 1) & 1);
+    if (softmax_barrier_and(ok)) {
+      tc_fence_after();
+      epilogue(pend);
+    } else {
+      failed = true;
+    }
+  }
+  if (failed && tid == 0) {
     *r.abort = 1;
     set_flag(r.flags, MQA_FLAG_PIPE_TIMEOUT);
   }
@@ -550,9 +659,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kSFull + s), 1);
       mbar_init(bar(C::kQFull + s), 1);
       mbar_init(bar(C::kQEmpty + s), 1);
-      mbar_init(bar(C::kOFree + s), 128);
+      mbar_init(bar(C::kOFree + s), 256);
     }
-    mbar_init(bar(C::kPFull), 128);
+    mbar_init(bar(C::kPFull), 256);
     mbar_init(bar(C::kOFull), 1);
     mbar_init(bar(C::kDone), 1);
     *r.abort = 0;
@@ -569,12 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // Inputs may come from the kernel before this one on the stream (the append).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const Sched sc = make_schedule<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags,
-                                           reinterpret_cast<int64_t*>(r.smem + C::kSched));
+  const WSched ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags,
+                                                     reinterpret_cast<int64_t*>(r.smem + C::kSched), kSegUnits);
+  const Sched& sc = ws.s;
   __syncthreads();
   if (warp >= 2) {   // zero the P buffer (it held the schedule scratch): pad columns stay zero
     uint4* p = reinterpret_cast<uint4*>(r.smem + C::kP);
-    for (int k = threadIdx.x - 64; k < int(C::kPBytes / 16); k += 128) p[k] = make_uint4(0, 0, 0, 0);
+    for (int k = threadIdx.x - 64; k < int(C::kPBytes / 16); k += 256) p[k] = make_uint4(0, 0, 0, 0);
   }
   tc_fence_before();
   __syncthreads();
@@ -583,18 +693,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (sc.t_begin < sc.t_end) {
     if (warp == 0) {
-      if (lane == 0) producer<NP, SK, SV, true>(a, sc, r, &tm_k, &tm_q);
-      else if (lane == 1) producer<NP, SK, SV, false>(a, sc, r, &tm_v, &tm_q);
+      if (lane == 0) producer<NP, SK, SV, true>(a, ws, r, &tm_k, &tm_q);
+      else if (lane == 1) producer<NP, SK, SV, false>(a, ws, r, &tm_v, &tm_q);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<NP, SK, SV>(a, sc, r);
+      if (lane == 0) mma_issuer<NP, SK, SV>(a, ws, r);
     } else {
-      softmax_epilogue<NP, SK, SV>(a, sc, r, warp, lane);
+      softmax_epilogue<NP, SK, SV>(a, ws, r, warp, lane);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(r.tmem, kTmemCols);
+  // The merge kernel may launch now (launching it earlier, to wait beside this
+  // grid, measured slower).
   asm volatile("griddepcontrol.launch_dependents;");
 }
 

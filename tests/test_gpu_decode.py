@@ -211,3 +211,36 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(binding.MqaError) as e:
         binding.decode(q, k, k, lens, 1.0, workspace=ws)
     assert e.value.status == binding.MQA_ERR_INVALID_ARG
+
+
+def test_workspace_reused_across_shapes():
+    """One workspace serves decodes of different shapes in turn; whatever an
+    earlier call left in it, every result matches the oracle."""
+    shapes = [(5, 32, 1, 700, 1, 700), (3, 64, 8, 500, 100, 500), (9, 16, 2, 300, 1, 300), (5, 32, 1, 700, 1, 700)]
+    need = max(binding.decode_workspace_size(b, h, g, 128) for b, h, g, *_ in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for n, (b, h, g, m, lo, hi) in enumerate(shapes):
+        wl = small("bf16", b, h, g, 128, m, lo, hi)
+        assert binding.decode_workspace_size(b, h, g, 128) <= ws.numel()
+        inp = host_inputs(wl, seed=40 + n, nan_tail=True)
+        for ctas in (0, 7):
+            o = binding.decode(dev(inp["q"], "bf16"), dev(inp["k"], "bf16"), dev(inp["v"], "bf16"),
+                               torch.from_numpy(inp["lens"]).cuda(), wl.scale, workspace=ws, num_ctas=ctas)
+            ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], inp["lens"], g, wl.scale)
+            assert_close(host64(o), ref, "bf16", f"shape {n} ctas {ctas}")
+
+
+@pytest.mark.parametrize("path", ["tcgen05", "simt"])
+def test_mixed_and_empty_lengths_many_ctas(path):
+    """Zero-length sequences (zero rows out), single-row sequences, long ones,
+    and more CTAs than tiles: the work partition must give every tile to
+    exactly one CTA and the merge must find every partial."""
+    wl = small("bf16", 12, 32 if path == "tcgen05" else 8, 1, 128, 900, 1, 1)
+    lens = np.array([0, 1, 900, 0, 129, 128, 2, 0, 700, 1, 255, 0], np.int32)
+    inp = host_inputs(wl, seed=77, nan_tail=False, lens=np.maximum(lens, 1))
+    for ctas in (0, 1, 5, 40, 300):
+        o = host64(binding.decode(dev(inp["q"], "bf16"), dev(inp["k"], "bf16"), dev(inp["v"], "bf16"),
+                                  torch.from_numpy(lens).cuda(), wl.scale, path=path, num_ctas=ctas))
+        ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, 1, wl.scale)
+        assert_close(o, ref, "bf16", f"{path} ctas={ctas}")
+        assert (o[lens == 0] == 0).all()

@@ -42,7 +42,7 @@ def _both(lib, wl, seed):
     dt = binding.MQA_BF16 if wl.dtype == "bf16" else binding.MQA_F32
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     ref = torch.empty((wl.b, wl.h, wl.d_v), dtype=q.dtype, device="cuda")
-    ws = torch.empty(binding.decode_workspace_size(wl.b, wl.h, wl.g, wl.d_v), dtype=torch.uint8, device="cuda")
+    ws = binding.new_workspace(wl.b, wl.h, wl.g, wl.d_v)
     st = lib.mqa_decode(_p(ref), _p(q), _p(K), _p(V), _p(lens), wl.b, wl.h, wl.g, wl.m_max, wl.d_k, wl.d_v,
                         wl.scale, dt, _p(ws), ws.numel(), None, stream)
     assert st == binding.MQA_OK
