@@ -11,7 +11,7 @@ from . import workloads  # noqa: F401
 
 _BINDING_NAMES = {
     "kv_append", "decode", "decode_workspace_size", "status_string", "lib", "MqaError",
-    "load_library", "DecodeOptions", "AppendPlan", "DecodePlan", "new_workspace",
+    "load_library", "DecodeOptions", "AppendPlan", "DecodePlan", "new_workspace", "decode_append",
 }
 
 

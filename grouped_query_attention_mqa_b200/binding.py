@@ -39,6 +39,9 @@ SIGNATURES = {
     "mqa_decode_ex": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_float, _c_int, _c_ptr, _c_size, _c_ptr, ctypes.POINTER(DecodeOptions),
                                _c_ptr]),
+    "mqa_decode_append": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int,
+                                   _c_int, _c_int, _c_int, _c_float, _c_int, _c_ptr, _c_size, _c_ptr,
+                                   ctypes.POINTER(DecodeOptions), _c_ptr]),
     "mqa_decode_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
                                     _c_int, _c_float, _c_int, _c_ptr, _c_ptr]),
     "mqa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -181,6 +184,15 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
     return out
 
 
+def decode_append(q, k_cache, v_cache, k_new, v_new, lens, scale, out=None, workspace=None, status_flags=None,
+                  path="auto", num_ctas=0, stream=None):
+    """One incremental step (mqa_decode_append): write k_new/v_new [b,g,d] at
+    row lens[b]-1 of the caches, then attend over lens[b] rows.  Returns o."""
+    plan = DecodePlan(q, k_cache, v_cache, lens, scale, out=out, workspace=workspace, status_flags=status_flags,
+                      path=path, num_ctas=num_ctas, stream=stream, k_new=k_new, v_new=v_new)
+    return plan.run()
+
+
 class AppendPlan:
     """mqa_kv_append with its arguments marshalled once, for loops that repeat
     the same call (a decode step on fixed buffers): ``run()`` is one C call."""
@@ -208,24 +220,37 @@ class DecodePlan:
     that writes ``self.out``."""
 
     def __init__(self, q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_flags=None, path="auto",
-                 num_ctas=0, stream=None):
+                 num_ctas=0, stream=None, k_new=None, v_new=None):
         import torch
-        _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags)
+        _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags, k_new, v_new)
         b, h, d_k = q.shape
         _, m_max, g, _ = k_cache.shape
         d_v = v_cache.shape[3]
+        if lens.dtype != torch.int32 or tuple(lens.shape) != (b,):
+            raise ValueError("lens must be int32 [b]")
+        if tuple(k_cache.shape) != (b, m_max, g, d_k) or tuple(v_cache.shape[:3]) != (b, m_max, g):
+            raise ValueError("DecodePlan: inconsistent cache shapes")
+        if (k_new is None) != (v_new is None):
+            raise ValueError("DecodePlan: give both k_new and v_new, or neither")
+        if k_new is not None and (tuple(k_new.shape) != (b, g, d_k) or tuple(v_new.shape) != (b, g, d_v)):
+            raise ValueError("DecodePlan: k_new/v_new must be [b,g,d]")
         if out is None:
             out = torch.empty((b, h, d_v), dtype=q.dtype, device=q.device)
         if workspace is None:
             workspace = new_workspace(b, h, g, d_v, device=q.device)
         self.out = out
         self._opts = DecodeOptions(PATHS[path], int(num_ctas))
-        self._keep = (q, k_cache, v_cache, lens, out, workspace, status_flags)
-        self._fn = lib().mqa_decode_ex
-        self._args = (_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), b, h, g, m_max, d_k, d_v,
-                      ctypes.c_float(scale), _dtype_code(q), _ptr(workspace),
-                      workspace.numel() * workspace.element_size(), _ptr(status_flags), ctypes.byref(self._opts),
-                      _stream_handle(stream))
+        self._keep = (q, k_cache, v_cache, lens, out, workspace, status_flags, k_new, v_new)
+        common = (ctypes.c_float(scale), _dtype_code(q), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                  _ptr(status_flags), ctypes.byref(self._opts), _stream_handle(stream))
+        if k_new is None:
+            self._fn = lib().mqa_decode_ex
+            self._args = (_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), b, h, g, m_max, d_k,
+                          d_v) + common
+        else:
+            self._fn = lib().mqa_decode_append
+            self._args = (_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(lens), b,
+                          h, g, m_max, d_k, d_v) + common
 
     def run(self):
         st = self._fn(*self._args)

@@ -352,6 +352,10 @@ struct DecodeArgs {
   const void* q;
   const void* k;
   const void* v;
+  // Fused append: when non-null, k_new/v_new [b, g, d] are written at row
+  // lens[b]-1 of the caches by the CTA that loads that row, before it loads it.
+  const void* k_new;
+  const void* v_new;
   const int32_t* lens;
   int b, h, g, m_max, d;
   int hq;

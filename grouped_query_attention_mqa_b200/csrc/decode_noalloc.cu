@@ -109,6 +109,8 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.q = q;
   a.k = k_cache;
   a.v = v_cache;
+  a.k_new = nullptr;
+  a.v_new = nullptr;
   a.lens = lens;
   a.b = b;
   a.h = h;

@@ -42,17 +42,32 @@ struct SimtLayout {
   }
 };
 
+// Stage the valid rows of a tile.  With the fused append (knew != nullptr)
+// the sequence's last tile holds its newest row: that row is taken from
+// knew/vnew, written into the cache and into the stage directly.
 template <typename T, int D>
 __device__ __forceinline__ void load_tile(unsigned char* ks, unsigned char* vs, const T* __restrict__ K,
-                                          const T* __restrict__ V, const TileCoord& tc, int g, int m_max) {
+                                          const T* __restrict__ V, const TileCoord& tc, int g, int m_max,
+                                          const T* __restrict__ knew, const T* __restrict__ vnew) {
   using L = SimtLayout<T, D>;
   const int n = tc.rows * L::kChunks;
   const int64_t row_base = (int64_t(tc.seq) * m_max + tc.row0) * g + tc.head;
+  const int new_row = (knew != nullptr && tc.k == tc.nb - 1) ? tc.rows - 1 : -1;
   for (int i = threadIdx.x; i < n; i += kThreads) {
     const int r = i / L::kChunks, c = i - r * L::kChunks;
     const int64_t off = (row_base + int64_t(r) * g) * D;        // element offset of the row
-    cp_async16(ks + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(K + off) + c * 16);
-    cp_async16(vs + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(V + off) + c * 16);
+    if (r == new_row) {
+      const int64_t src = (int64_t(tc.seq) * g + tc.head) * D;
+      const uint4 kv = reinterpret_cast<const uint4*>(knew + src)[c];
+      const uint4 vv = reinterpret_cast<const uint4*>(vnew + src)[c];
+      reinterpret_cast<uint4*>(const_cast<T*>(K) + off)[c] = kv;
+      reinterpret_cast<uint4*>(const_cast<T*>(V) + off)[c] = vv;
+      *reinterpret_cast<uint4*>(ks + r * L::kRowBytes + c * 16) = kv;
+      *reinterpret_cast<uint4*>(vs + r * L::kRowBytes + c * 16) = vv;
+    } else {
+      cp_async16(ks + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(K + off) + c * 16);
+      cp_async16(vs + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(V + off) + c * 16);
+    }
   }
 }
 
@@ -127,6 +142,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   const T* __restrict__ Q = static_cast<const T*>(a.q);
   const T* __restrict__ K = static_cast<const T*>(a.k);
   const T* __restrict__ V = static_cast<const T*>(a.v);
+  const T* __restrict__ KN = static_cast<const T*>(a.k_new);
+  const T* __restrict__ VN = static_cast<const T*>(a.v_new);
   T* __restrict__ O = static_cast<T*>(a.o);
   const int hq = a.hq, g = a.g;
   const float qscale = a.scale * kLog2e;
@@ -144,7 +161,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   cursor_seek(cur, a.lens, g, a.m_max, kTile, sc.t_begin);
   {
     const TileCoord t0 = tile_coord(cur, g, kTile, sc.t_begin);
-    load_tile<T, D>(stage, stage + 2 * kStageBytes, K, V, t0, g, a.m_max);
+    load_tile<T, D>(stage, stage + 2 * kStageBytes, K, V, t0, g, a.m_max, KN, VN);
     cp_async_commit();
   }
 
@@ -176,7 +193,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
       cursor_seek(nxt, a.lens, g, a.m_max, kTile, t + 1);
       const TileCoord tn = tile_coord(nxt, g, kTile, t + 1);
       load_tile<T, D>(stage + (st ^ 1) * kStageBytes, stage + (2 + (st ^ 1)) * kStageBytes, K, V, tn, g,
-                      a.m_max);
+                      a.m_max, KN, VN);
     }
     cp_async_commit();
     cp_async_wait1();

@@ -15,6 +15,11 @@
 // of the group reads the same staged tile — the bandwidth saving MQA is for.
 // S and O live in tensor memory; O accumulates over all tiles of a segment.
 //
+// With the fused append (k_new/v_new given) the producer that owns a
+// sequence's last tile first writes the step's new K (or V) row into the cache
+// at row lens-1 and then loads the tile, so the row is both stored for later
+// steps and attended to now.
+//
 // Roles (one CTA per SM, persistent over an even share of all tiles):
 //   warp 0, lane 0      TMA producer of Q (per segment) and of K tiles into a
 //                       ring of SK stages; a K stage is released as soon as
@@ -254,6 +259,22 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     if (i >= S && !wait_bar(r, bar(kEmpty + st), uint32_t((i / S) - 1) & 1)) break;
     const int row = w.tc.seq * a.m_max + w.tc.row0;
     const uint32_t dst = r.sbase + kRing + st * kTileBytes;
+    if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1) {
+      // Fused append: this tile holds the sequence's newest row (lens-1);
+      // write it into the cache first, then order that store before the
+      // tensor-memory-access read of the same row.
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(kIsK ? a.k_new : a.v_new) +
+                                                        (int64_t(w.tc.seq) * a.g + w.tc.head) * kD);
+      uint4* cache = reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(
+          static_cast<const __nv_bfloat16*>(kIsK ? a.k : a.v) +
+          ((int64_t(w.tc.seq) * a.m_max + (w.len - 1)) * a.g + w.tc.head) * kD));
+      uint4 tmp[kD / 8];
+#pragma unroll
+      for (int c = 0; c < kD / 8; ++c) tmp[c] = __ldg(src + c);
+#pragma unroll
+      for (int c = 0; c < kD / 8; ++c) cache[c] = tmp[c];
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
     mbar_expect_tx(bar(kFull + st), kTileBytes);
     tma_load_3d(dst, tm_kv, bar(kFull + st), 0, w.tc.head, row, pol);
     tma_load_3d(dst + kHalfBytes, tm_kv, bar(kFull + st), 64, w.tc.head, row, pol);

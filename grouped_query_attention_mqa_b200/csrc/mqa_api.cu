@@ -62,10 +62,15 @@ size_t mqa_decode_workspace_size(int b, int h, int g, int d_v) {
   return workspace_bytes(b, g, h / g, d_v);
 }
 
-mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens,
-                           int b, int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype,
-                           void* workspace, size_t workspace_bytes_given, int32_t* status_flags,
-                           const mqa_decode_opts_t* opts, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// mqa_decode_ex, and with k_new/v_new the fused append + decode.
+mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void* v_cache, const void* k_new,
+                         const void* v_new, const int32_t* lens, int b, int h, int g, int m_max, int d_k, int d_v,
+                         float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes_given,
+                         int32_t* status_flags, const mqa_decode_opts_t* opts, cudaStream_t stream) {
   if (b < 0 || h < 1 || g < 1 || h % g != 0 || m_max < 1 || d_k < 1 || d_v < 1 || !valid_dtype(dtype) ||
       !std::isfinite(scale))
     return MQA_ERR_INVALID_ARG;
@@ -74,6 +79,8 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
   if (opts && (opts->num_ctas < 0 || opts->num_ctas > kMaxCtas)) return MQA_ERR_INVALID_ARG;
   if (b == 0) return MQA_OK;
   if (!o || !q || !k_cache || !v_cache || !lens || !workspace) return MQA_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return MQA_ERR_INVALID_ARG;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return MQA_ERR_INVALID_ARG;
   if (!aligned16(o) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(lens) ||
       !aligned256(workspace))
     return MQA_ERR_INVALID_ARG;
@@ -104,6 +111,8 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
   a.q = q;
   a.k = k_cache;
   a.v = v_cache;
+  a.k_new = k_new;
+  a.v_new = v_new;
   a.lens = lens;
   a.b = b;
   a.h = h;
@@ -125,11 +134,33 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
   return MQA_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens,
+                           int b, int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes_given, int32_t* status_flags,
+                           const mqa_decode_opts_t* opts, cudaStream_t stream) {
+  return decode_impl(o, q, k_cache, v_cache, nullptr, nullptr, lens, b, h, g, m_max, d_k, d_v, scale, dtype,
+                     workspace, workspace_bytes_given, status_flags, opts, stream);
+}
+
 mqa_status_t mqa_decode(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int b,
                         int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype, void* workspace,
                         size_t workspace_bytes_given, int32_t* status_flags, cudaStream_t stream) {
-  return mqa_decode_ex(o, q, k_cache, v_cache, lens, b, h, g, m_max, d_k, d_v, scale, dtype, workspace,
-                       workspace_bytes_given, status_flags, nullptr, stream);
+  return decode_impl(o, q, k_cache, v_cache, nullptr, nullptr, lens, b, h, g, m_max, d_k, d_v, scale, dtype,
+                     workspace, workspace_bytes_given, status_flags, nullptr, stream);
+}
+
+mqa_status_t mqa_decode_append(void* o, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                               const void* v_new, const int32_t* lens, int b, int h, int g, int m_max, int d_k,
+                               int d_v, float scale, mqa_dtype_t dtype, void* workspace,
+                               size_t workspace_bytes_given, int32_t* status_flags, const mqa_decode_opts_t* opts,
+                               cudaStream_t stream) {
+  if (b > 0 && (k_new == nullptr || v_new == nullptr)) return MQA_ERR_INVALID_ARG;
+  return decode_impl(o, q, k_cache, v_cache, k_new, v_new, lens, b, h, g, m_max, d_k, d_v, scale, dtype, workspace,
+                     workspace_bytes_given, status_flags, opts, stream);
 }
 
 }  // extern "C"

@@ -160,6 +160,31 @@ MQA_API mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, 
                            float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes,
                            int32_t* status_flags, const mqa_decode_opts_t* opts, cudaStream_t stream);
 
+/*
+ * mqa_decode_append — one whole incremental step: append, then attend.
+ *
+ * Source: the velog paper review, §3 MultiquerySelfAttentionIncremental:
+ * new_K = concat(prev_K, k_new), new_V likewise, then the attention of
+ * mqa_decode over new_K/new_V.  Here lens[b] counts the rows after the
+ * append, so the step's K/V row goes to row lens[b]-1.  Same result as
+ * mqa_kv_append(pos = lens-1) followed by mqa_decode(lens), in one launch:
+ * the CTA that loads a sequence's last tile first writes the new row into the
+ * cache, then attends over it.
+ *
+ *   k_cache, v_cache  device [b, m_max, g, d]   read, and row lens[b]-1 written
+ *   k_new, v_new      device [b, g, d]          read
+ *   other arguments as for mqa_decode_ex; lens outside [1, m_max] are clamped
+ *   and flagged as there (the row then goes to the clamped length minus one;
+ *   a sequence whose clamped length is 0 writes nothing and outputs zeros).
+ * Errors as for mqa_decode_ex, plus MQA_ERR_INVALID_ARG for NULL or
+ * misaligned k_new / v_new.
+ */
+MQA_API mqa_status_t mqa_decode_append(void* o, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                                       const void* v_new, const int32_t* lens, int b, int h, int g, int m_max,
+                                       int d_k, int d_v, float scale, mqa_dtype_t dtype, void* workspace,
+                                       size_t workspace_bytes, int32_t* status_flags,
+                                       const mqa_decode_opts_t* opts, cudaStream_t stream);
+
 /* Size of the device array that mqa_decode_noalloc uses as its scratch. */
 #define MQA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
