@@ -136,6 +136,31 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ ranks
+
+def rank_seed(rank: int) -> int:
+    """Each rank decodes its own independent batch (weak scaling)."""
+    return SEED + rank
+
+
+def reduce_over_ranks(values, device):
+    """Max over ranks of each timing: the slowest rank sets the job's time.
+    Runs on whatever process group is initialised (NCCL on GPUs, gloo in the
+    CPU tests); returns the values unchanged on a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(world: int, b: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job query-tokens/s: every rank decodes b new tokens per step."""
+    return world * b * steps / (elapsed_ms / 1e3)
+
+
 # ------------------------------------------------------------------ GPU side
 
 class ClockSampler:
@@ -262,7 +287,7 @@ def run_ours(args):
     cache_bytes = wl.b * wl.m_max * wl.g * (wl.d_k + wl.d_v) * wl.elem_bytes
     # enough copies that >= 2 other steps (and >= 3x L2 of cache) pass between two uses of one copy
     copies = max(3, min(8, -(-3 * L2_BYTES // cache_bytes) + 1))
-    inp = device_inputs(wl, seed=SEED + rank, device="cuda", copies=copies)
+    inp = device_inputs(wl, seed=rank_seed(rank), device="cuda", copies=copies)
     lens_np = inp["lens"]
     lens = torch.from_numpy(lens_np).cuda()
     out = torch.empty((b, h, wl.d_v), dtype=inp["q"].dtype, device="cuda")
@@ -303,12 +328,9 @@ def run_ours(args):
     elapsed_ms = start.elapsed_time(end)
     dec_ms = [a.elapsed_time(z) for a, z in ev_dec]
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    if world > 1:
-        t = torch.tensor([elapsed_ms, dec_avg_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_avg_ms = float(t[0]), float(t[1])
+    elapsed_ms, dec_avg_ms = reduce_over_ranks([elapsed_ms, dec_avg_ms], "cuda")
     ms_per_step = elapsed_ms / K
-    value = world * b * K / (elapsed_ms / 1e3)
+    value = job_value(world, b, K, elapsed_ms)
 
     # end to end through the public API: pinned host inputs copied in, the
     # step's output copied out, every step
@@ -345,12 +367,8 @@ def run_ours(args):
         e2e_step(i)
     e2.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * b * E / (e2e_ms / 1e3)
+    e2e_ms = reduce_over_ranks([s2.elapsed_time(e2)], "cuda")[0]
+    e2e_value = job_value(world, b, E, e2e_ms)
 
     alg_bytes = decode_algorithmic_bytes(wl, lens_np) + append_algorithmic_bytes(wl)
     peak, peak_kind = peaks()
