@@ -60,6 +60,7 @@ constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
 constexpr int kSegUnits = 6;                 // cost of entering a segment, in quarter tiles (partition weight)
+constexpr int kLensCache = 64;               // clamped lengths of a CTA's first sequences, kept in shared memory
 constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O double buffer at [128, 256)
 constexpr uint32_t kOCol = 128;
 constexpr uint32_t kMaxDynSmem = 232448;     // 227 KB opt-in limit per CTA
@@ -87,7 +88,9 @@ struct TcCfg {
   static constexpr uint32_t kRedL = kAlpha + NP * 4;             // [4][NP] f32: per-warp head sums
   static constexpr uint32_t kLinv = kRedL + 4 * NP * 4;          // [2][NP]: 1 / l per segment parity
   static constexpr uint32_t kLse = kLinv + 2 * NP * 4;           // [2][NP]: log2-sum-exp per segment parity
-  static constexpr uint32_t kEnd = kLse + 2 * NP * 4;
+  static constexpr uint32_t kLens = kLse + 2 * NP * 4;          // [kLensCache] clamped lengths from seq0
+  static constexpr uint32_t kKIssued = kLens + kLensCache * 4;   // K tiles issued so far (V producer trails it)
+  static constexpr uint32_t kEnd = kKIssued + 16;
   static constexpr uint32_t kAlloc = kEnd + 1024;             // room to align the base to 1024 bytes
   static constexpr uint32_t kSched = kP;                      // start-up scratch, before P is zeroed
   static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kQBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
@@ -155,7 +158,18 @@ struct Roles {
   uint32_t tmem;
   volatile int* abort;
   int32_t* flags;
+  const int* lens_s;         // clamped lens[seq0 + i], i < kLensCache (global memory beyond that)
+  int seq0;
 };
+
+// Clamped length of sequence s: from shared memory for the CTA's first
+// sequences.  Under the start-up flood of TMA loads a dependent global load
+// here would stall the role that needs it for thousands of cycles.
+__device__ __forceinline__ int seq_len(const DecodeArgs& a, const Roles& r, int s) {
+  const int i = s - r.seq0;
+  if (i >= 0 && i < kLensCache) return r.lens_s[i];
+  return clamp_len(__ldg(a.lens + s), a.m_max, nullptr, false);
+}
 
 __device__ __forceinline__ bool wait_bar(const Roles& r, uint32_t bar, uint32_t parity) {
   if (mbar_wait(bar, parity, kTimeoutNs)) return true;
@@ -176,17 +190,18 @@ struct TileWalk {
   int sidx;                  // segment number within this CTA
   TileCoord tc;
   bool first, last;
-  __device__ TileWalk(const DecodeArgs& a, const WSched& ws) : t(ws.s.t_begin - 1), sidx(-1) {
+  const Roles* rr;
+  __device__ TileWalk(const DecodeArgs& a, const WSched& ws, const Roles& r) : t(ws.s.t_begin - 1), sidx(-1), rr(&r) {
     seq = ws.s.seq;
     base = ws.s.seq_base;
     ubase = ws.seq_ubase;
-    len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
+    len = seq_len(a, r, seq);
     nb = tiles_of(len, kTile);
     while (ws.s.t_begin >= base + int64_t(a.g) * nb) {   // the first tile may lie in a later sequence
       base += int64_t(a.g) * nb;
       ubase += seq_units(nb, a.g, kSegUnits);
       ++seq;
-      len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
+      len = seq_len(a, r, seq);
       nb = tiles_of(len, kTile);
     }
     const int64_t rel = ws.s.t_begin - base;
@@ -203,7 +218,7 @@ struct TileWalk {
         ubase += seq_units(nb, a.g, kSegUnits);
         do {
           ++seq;
-          len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
+          len = seq_len(a, *rr, seq);
           nb = tiles_of(len, kTile);
         } while (nb == 0);
       }
@@ -238,7 +253,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
   constexpr uint32_t kRing = kIsK ? C::kK : C::kV;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  TileWalk w(a, ws);
+  TileWalk w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t i = 0;
   int q_issued = -1;
@@ -257,6 +272,13 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     }
     const int st = int(i % S);
     if (i >= S && !wait_bar(r, bar(kEmpty + st), uint32_t((i / S) - 1) & 1)) break;
+    if (!kIsK) {   // never run ahead of the K producer: the loads go out K(0), V(0), K(1), ...
+      volatile int* k_issued = reinterpret_cast<volatile int*>(r.smem + C::kKIssued);
+      uint32_t polls = 0;
+      while (*k_issued <= i && !*r.abort) {
+        if ((++polls & 1023u) == 0 && polls > (1u << 24)) break;   // cannot stall for good: K gives up on abort
+      }
+    }
     const int row = w.tc.seq * a.m_max + w.tc.row0;
     const uint32_t dst = r.sbase + kRing + st * kTileBytes;
     if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1) {
@@ -278,6 +300,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     mbar_expect_tx(bar(kFull + st), kTileBytes);
     tma_load_3d(dst, tm_kv, bar(kFull + st), 0, w.tc.head, row, pol);
     tma_load_3d(dst + kHalfBytes, tm_kv, bar(kFull + st), 64, w.tc.head, row, pol);
+    if (kIsK) *reinterpret_cast<volatile int*>(r.smem + C::kKIssued) = int(i + 1);
   }
   // Drain: every copy this thread issued has landed before the CTA can exit.
   for (int64_t j = (i - S > 0 ? i - S : 0); j < i; ++j)
@@ -301,7 +324,7 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int64_t n = sc.t_end - sc.t_begin;
-  TileWalk wq(a, ws), wp(a, ws);   // walkers for the S stream and the O stream
+  TileWalk wq(a, ws, r), wp(a, ws, r);   // walkers for the S stream and the O stream
   const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);           // K-major, rows of 128 B
   const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
   const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
@@ -410,7 +433,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
   float lpart[CPT];                                // this row's share of the per-head sums
   float sv[CPT];                                   // this row's scaled logits (log2 units)
   float mr[CPT];                                   // reference max per head, mirrored from smem
-  TileWalk w(a, ws);
+  TileWalk w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t pv_waited = -1;
   bool failed = false;
@@ -702,6 +725,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WSched ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags,
                                                      reinterpret_cast<int64_t*>(r.smem + C::kSched), kSegUnits);
   const Sched& sc = ws.s;
+  r.seq0 = sc.seq;
+  r.lens_s = reinterpret_cast<const int*>(r.smem + C::kLens);
+  if (threadIdx.x < kLensCache && sc.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them
+    reinterpret_cast<int*>(r.smem + C::kLens)[threadIdx.x] =
+        clamp_len(__ldg(a.lens + sc.seq + threadIdx.x), a.m_max, nullptr, false);
+  if (threadIdx.x == 0) *reinterpret_cast<int*>(r.smem + C::kKIssued) = 0;
   __syncthreads();
   if (warp >= 2) {   // zero the P buffer (it held the schedule scratch): pad columns stay zero
     uint4* p = reinterpret_cast<uint4*>(r.smem + C::kP);
@@ -811,8 +840,8 @@ int tc_ctas_per_sm(int) { return 1; }
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) || int64_t(a.b) * a.h >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
-  if (a.hq <= 16) return launch_np<16, 3, 3>(a, stream);
-  if (a.hq <= 32) return launch_np<32, 3, 3>(a, stream);
+  if (a.hq <= 16) return launch_np<16, 2, 3>(a, stream);
+  if (a.hq <= 32) return launch_np<32, 2, 3>(a, stream);
   if (a.hq <= 64) return launch_np<64, 2, 3>(a, stream);
   return cudaErrorInvalidValue;
 }
