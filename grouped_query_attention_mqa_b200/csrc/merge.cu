@@ -22,6 +22,8 @@ constexpr int kMergeThreads = 128;
 template <typename T>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a, int heads_per_cta) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The next step's decode may launch and set up while the merge runs.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int hq = a.hq, D = a.d;
   const int chunks = (hq + heads_per_cta - 1) / heads_per_cta;
   const int64_t s = blockIdx.x / chunks;
