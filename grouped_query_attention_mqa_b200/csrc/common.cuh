@@ -190,6 +190,7 @@ struct WSched {
   Sched s;
   int64_t wtotal;     // W: units over all segments
   int64_t seq_ubase;  // first unit of sequence s.seq
+  int pre;            // leading tiles whose loads the schedule already issued
 };
 
 __device__ __forceinline__ int64_t seq_units(int nb, int g, int xw) {
@@ -255,6 +256,7 @@ __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b
   ws.s.seq = 0;
   ws.s.seq_base = 0;
   ws.seq_ubase = 0;
+  ws.pre = 0;
   if (cta >= ws.s.active) return ws;   // uniform across the CTA
   const int64_t u0 = (int64_t(cta) * W) / ws.s.active;
   const int64_t u1 = ((int64_t(cta) + 1) * W) / ws.s.active;
@@ -291,6 +293,105 @@ __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b
   ws.s.seq_base = out[2];
   ws.seq_ubase = out[3];
   ws.s.t_end = u1 == W ? T : out[4];
+  ws.pre = 0;
+  return ws;
+}
+
+// The same weighted partition when every sequence has a thread (b <= NT) and
+// the unit total stays below 2^31 (checked by small_schedule_fits): each thread
+// loads one length, which it also leaves in lens_tab[s] (clamped) for the rest
+// of the kernel; the tile and unit counts are scanned together as one 64-bit
+// word (high and low halves, neither can carry), and the range ends are found
+// with 32-bit arithmetic.  Two block barriers.  `red` needs NT/32 + 8 int64.
+// The thread that finds the CTA's first tile calls
+// on_first(seq, head, k, own, len, nb) at once, with `own` >= 1 tiles of that
+// segment from tile k on belonging to the CTA; it returns how many of them it
+// has started to load (WSched::pre).  Code that runs once per launch executes
+// at instruction-fetch speed, so this gets the first loads out well before a
+// separate role would reach them.
+__device__ __forceinline__ bool small_schedule_fits(int b, int g, int m_max, int tile, int nt, int xw) {
+  return b <= nt && int64_t(b) * g * (xw + 4 * (int64_t(m_max) + tile - 1) / tile) < (int64_t(1) << 31);
+}
+
+template <int NT, typename OnFirst>
+__device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile, int grid,
+                                      int cta, int32_t* flags, int64_t* red, int xw, int* lens_tab,
+                                      OnFirst&& on_first) {
+  static_assert(NT % 32 == 0, "whole warps");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int len = 0;
+  if (tid < b) {
+    len = clamp_len(__ldg(lens + tid), m_max, flags, cta == 0);
+    lens_tab[tid] = len;
+  }
+  const int nb = tiles_of(len, tile);
+  const int my_t = g * nb;
+  const int my_u = nb > 0 ? g * (xw + 4 * nb) : 0;
+  uint64_t x = (uint64_t(uint32_t(my_t)) << 32) | uint32_t(my_u);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  uint64_t* wsum = reinterpret_cast<uint64_t*>(red);   // [NT/32]
+  int64_t* out = red + NT / 32;
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  uint64_t tot = 0, before = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const uint64_t v = wsum[w];
+    tot += v;
+    if (w < warp) before += v;
+  }
+  const uint64_t incl = before + x;
+  const int T = int(tot >> 32), W = int(uint32_t(tot));
+  const int excl_t = int(incl >> 32) - my_t, excl_u = int(uint32_t(incl)) - my_u;
+  WSched ws;
+  ws.s.total = T;
+  ws.wtotal = W;
+  const int cap = W / (xw + 4);
+  ws.s.active = cap < grid ? cap : grid;
+  ws.s.t_begin = ws.s.t_end = 0;
+  ws.s.seq = 0;
+  ws.s.seq_base = 0;
+  ws.seq_ubase = 0;
+  ws.pre = 0;
+  if (cta >= ws.s.active) return ws;   // uniform across the CTA
+  // c*W/A without a 64-bit product: W = q*A + rm and c*rm < A*A
+  const int q = W / ws.s.active, rm = W - q * ws.s.active;
+  const int u0 = cta * q + (cta * rm) / ws.s.active;
+  const int u1 = (cta + 1) * q + ((cta + 1) * rm) / ws.s.active;
+  const int seglen = xw + 4 * nb;
+  auto first_tile = [&](int u) {   // tiles of this thread's sequence whose start unit is below u
+    const int rel = u - excl_u;
+    const int j = rel / seglen, off = rel - j * seglen;
+    return excl_t + j * nb + (off <= xw ? 0 : (off - xw + 3) / 4);
+  };
+  if (u1 < W && u1 >= excl_u && u1 < excl_u + my_u) out[4] = first_tile(u1);
+  if (u0 >= excl_u && u0 < excl_u + my_u) {
+    const int rel = u0 - excl_u;
+    const int j = rel / seglen, off = rel - j * seglen;
+    const int k = off <= xw ? 0 : (off - xw + 3) / 4;
+    out[0] = excl_t + j * nb + k;
+    out[1] = tid;
+    out[2] = excl_t;
+    out[3] = excl_u;
+    int started = 0;
+    if (k < nb) {   // tile k of segment j exists; the CTA owns its tiles whose start unit is below u1
+      const int lim = u1 - (excl_u + j * seglen + xw);
+      const int kend = min(nb, lim <= 0 ? 0 : (lim + 3) / 4);
+      if (kend > k) started = on_first(tid, j, k, kend - k, len, nb);
+    }
+    out[5] = started;
+  }
+  __syncthreads();
+  ws.s.t_begin = out[0];
+  ws.s.seq = int(out[1]);
+  ws.s.seq_base = out[2];
+  ws.seq_ubase = out[3];
+  ws.s.t_end = u1 == W ? T : out[4];
+  ws.pre = int(out[5]);
   return ws;
 }
 

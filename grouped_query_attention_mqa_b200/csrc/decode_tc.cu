@@ -24,14 +24,18 @@
 //   warp 0, lane 0      TMA producer of Q (per segment) and of K tiles into a
 //                       ring of SK stages; a K stage is released as soon as
 //                       the S product that reads it has completed.
-//   warp 0, lane 1      TMA producer of V tiles into a ring of SV stages,
-//                       released when the P.V product has completed.  Both
-//                       rings use L2 evict-first: each byte is read once.
+//   warp 10, lane 0     TMA producer of V tiles into a ring of SV stages,
+//                       released when the P.V product has completed; it
+//                       never runs ahead of the K producer.  Both rings use
+//                       L2 evict-first: each byte is read once.  The two
+//                       producers sit in different warps because the waits of
+//                       two diverged threads of one warp are serialised.
 //   warp 1, lane 0      MMA issuer: S(i+1) = K Q^T while P(i) is being made,
 //                       then O += V^T P(i); completions are signalled with
 //                       tcgen05.commit on mbarriers.
-//   warps 2-5           softmax and epilogue, one cache row (then one output
-//                       column) per thread.  The reference max per head is set
+//   warps 2-9           softmax and epilogue in two column groups of four
+//                       warps: one cache row (then one output column) and
+//                       half of the heads per thread.  The reference max per head is set
 //                       from the first tile of a segment and only moved when
 //                       some logit exceeds it by more than 8 (a factor 256 in
 //                       exp2); only then do the warps reduce column maxima and
@@ -53,14 +57,15 @@ using namespace sm100;
 
 constexpr int kTile = 128;                   // cache rows per tile (the MMA M)
 constexpr int kD = 128;                      // head size
-constexpr int kThreads = 320;             // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kThreads = 352;                // warp 0 K/Q loads, warp 1 MMA, warps 2-9 softmax, warp 10 V loads
+constexpr int kVWarp = 10;
 constexpr int kNpv = 64;                     // N of the P.V product (P padded with zero columns)
 constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte swizzle column
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
 constexpr int kSegUnits = 6;                 // cost of entering a segment, in quarter tiles (partition weight)
-constexpr int kLensCache = 64;               // clamped lengths of a CTA's first sequences, kept in shared memory
+constexpr int kLensCache = kThreads;         // clamped lengths kept in shared memory (all of them when b <= kThreads)
 constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O double buffer at [128, 256)
 constexpr uint32_t kOCol = 128;
 constexpr uint32_t kMaxDynSmem = 232448;     // 227 KB opt-in limit per CTA
@@ -90,12 +95,14 @@ struct TcCfg {
   static constexpr uint32_t kLse = kLinv + 2 * NP * 4;           // [2][NP]: log2-sum-exp per segment parity
   static constexpr uint32_t kLens = kLse + 2 * NP * 4;          // [kLensCache] clamped lengths from seq0
   static constexpr uint32_t kKIssued = kLens + kLensCache * 4;   // K tiles issued so far (V producer trails it)
-  static constexpr uint32_t kEnd = kKIssued + 16;
+  static constexpr uint32_t kSched = kKIssued + 16;            // start-up scratch of the schedule
+  static constexpr uint32_t kEnd = kSched + 256;
   static constexpr uint32_t kAlloc = kEnd + 1024;             // room to align the base to 1024 bytes
-  static constexpr uint32_t kSched = kP;                      // start-up scratch, before P is zeroed
   static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kQBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kAlloc <= kMaxDynSmem, "shared memory budget");
-  static_assert((2 * (kThreads / 32) + 8) * 8 <= kPBytes, "schedule scratch fits in P");
+  static_assert((2 * (kThreads / 32) + 8) * 8 <= 256, "schedule scratch");
+  static_assert(kSched % 8 == 0, "schedule scratch alignment");
+  static_assert(kLens % 4 == 0, "lens table alignment");
 };
 
 __device__ __forceinline__ void named_barrier_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -159,12 +166,13 @@ struct Roles {
   volatile int* abort;
   int32_t* flags;
   const int* lens_s;         // clamped lens[seq0 + i], i < kLensCache (global memory beyond that)
-  int seq0;
+  int seq0;                  // 0 when the whole batch is in the table
 };
 
-// Clamped length of sequence s: from shared memory for the CTA's first
-// sequences.  Under the start-up flood of TMA loads a dependent global load
-// here would stall the role that needs it for thousands of cycles.
+// Clamped length of sequence s: from shared memory (the whole batch when it
+// has at most kLensCache sequences, else the CTA's first ones).  Under the
+// start-up flood of TMA loads a dependent global load here would stall the
+// role that needs it for thousands of cycles.
 __device__ __forceinline__ int seq_len(const DecodeArgs& a, const Roles& r, int s) {
   const int i = s - r.seq0;
   if (i >= 0 && i < kLensCache) return r.lens_s[i];
@@ -204,9 +212,9 @@ struct TileWalk {
       len = seq_len(a, r, seq);
       nb = tiles_of(len, kTile);
     }
-    const int64_t rel = ws.s.t_begin - base;
-    head = int(rel / nb);
-    k = int(rel - int64_t(head) * nb) - 1;   // next() advances to the first tile
+    const int rel = int(ws.s.t_begin - base);   // < g * nb
+    head = rel / nb;
+    k = rel - head * nb - 1;                     // next() advances to the first tile
   }
   __device__ void next(const DecodeArgs& a, const Sched& sc) {
     ++t;
@@ -241,6 +249,58 @@ struct TileWalk {
   }
 };
 
+// Fused append: write the step's new row of (sequence, K/V head) into the
+// cache at row len-1, then order that store before the tensor-memory-access
+// read of the same row.
+__device__ __forceinline__ void append_new_row(const DecodeArgs& a, bool is_k, int seq, int head, int len) {
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(is_k ? a.k_new : a.v_new) +
+                                                    (int64_t(seq) * a.g + head) * kD);
+  uint4* cache = reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(
+      static_cast<const __nv_bfloat16*>(is_k ? a.k : a.v) + ((int64_t(seq) * a.m_max + (len - 1)) * a.g + head) * kD));
+  uint4 tmp[kD / 8];
+#pragma unroll
+  for (int c = 0; c < kD / 8; ++c) tmp[c] = __ldg(src + c);
+#pragma unroll
+  for (int c = 0; c < kD / 8; ++c) cache[c] = tmp[c];
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Loads of the CTA's first tiles, issued by the schedule thread that finds
+// them: Q of the segment into Q buffer 0 and the first min(2, own) K and V
+// tiles into stages 0 and 1 (K before V, as the producers order them).
+// Returns the number of tiles started; the producers skip those.
+template <int NP, int SK, int SV>
+__device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                         const CUtensorMap* tm_q, int seq, int head, int k0, int own, int len, int nb) {
+  using C = TcCfg<NP, SK, SV>;
+  static_assert(SK >= 2 && SV >= 2, "two stages of each ring");
+  auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
+  const uint64_t pol = l2_evict_first_policy();
+  const int qrow = seq * a.h + head * a.hq;
+  const uint32_t qdst = r.sbase + C::kQ;
+  mbar_expect_tx(bar(C::kQFull), 2 * NP * 128);
+  tma_load_2d(qdst, tm_q, bar(C::kQFull), 0, qrow);
+  tma_load_2d(qdst + NP * 128, tm_q, bar(C::kQFull), 64, qrow);
+  const int npre = own < 2 ? own : 2;
+  for (int i = 0; i < npre; ++i) {
+    const int k = k0 + i;
+    if (a.k_new != nullptr && k == nb - 1) {
+      append_new_row(a, true, seq, head, len);
+      append_new_row(a, false, seq, head, len);
+    }
+    const int row = seq * a.m_max + k * kTile;
+    const uint32_t kdst = r.sbase + C::kK + i * kTileBytes;
+    mbar_expect_tx(bar(C::kKFull + i), kTileBytes);
+    tma_load_3d(kdst, tm_k, bar(C::kKFull + i), 0, head, row, pol);
+    tma_load_3d(kdst + kHalfBytes, tm_k, bar(C::kKFull + i), 64, head, row, pol);
+    const uint32_t vdst = r.sbase + C::kV + i * kTileBytes;
+    mbar_expect_tx(bar(C::kVFull + i), kTileBytes);
+    tma_load_3d(vdst, tm_v, bar(C::kVFull + i), 0, head, row, pol);
+    tma_load_3d(vdst + kHalfBytes, tm_v, bar(C::kVFull + i), 64, head, row, pol);
+  }
+  return npre;
+}
+
 // K ring and the per-segment Q (kIsK), or the V ring.
 template <int NP, int SK, int SV, bool kIsK>
 __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, const CUtensorMap* tm_kv,
@@ -257,9 +317,17 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t i = 0;
   int q_issued = -1;
+  const int64_t pre = ws.pre;   // tiles (and the first Q) the schedule already loads
   for (; i < n; ++i) {
     w.next(a, sc);
     if (*r.abort) break;
+    if (i < pre) {
+      if (kIsK) {
+        q_issued = 0;
+        *reinterpret_cast<volatile int*>(r.smem + C::kKIssued) = int(i + 1);
+      }
+      continue;
+    }
     if (kIsK && w.first) {
       const int qb = w.sidx & 1;
       if (w.sidx >= 2 && !wait_bar(r, bar(C::kQEmpty + qb), ((w.sidx >> 1) - 1) & 1)) break;
@@ -281,22 +349,8 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     }
     const int row = w.tc.seq * a.m_max + w.tc.row0;
     const uint32_t dst = r.sbase + kRing + st * kTileBytes;
-    if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1) {
-      // Fused append: this tile holds the sequence's newest row (lens-1);
-      // write it into the cache first, then order that store before the
-      // tensor-memory-access read of the same row.
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(kIsK ? a.k_new : a.v_new) +
-                                                        (int64_t(w.tc.seq) * a.g + w.tc.head) * kD);
-      uint4* cache = reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(
-          static_cast<const __nv_bfloat16*>(kIsK ? a.k : a.v) +
-          ((int64_t(w.tc.seq) * a.m_max + (w.len - 1)) * a.g + w.tc.head) * kD));
-      uint4 tmp[kD / 8];
-#pragma unroll
-      for (int c = 0; c < kD / 8; ++c) tmp[c] = __ldg(src + c);
-#pragma unroll
-      for (int c = 0; c < kD / 8; ++c) cache[c] = tmp[c];
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-    }
+    if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1)   // this tile holds the sequence's newest row
+      append_new_row(a, kIsK, w.tc.seq, w.tc.head, w.len);
     mbar_expect_tx(bar(kFull + st), kTileBytes);
     tma_load_3d(dst, tm_kv, bar(kFull + st), 0, w.tc.head, row, pol);
     tma_load_3d(dst + kHalfBytes, tm_kv, bar(kFull + st), 64, w.tc.head, row, pol);
@@ -433,6 +487,11 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
   float lpart[CPT];                                // this row's share of the per-head sums
   float sv[CPT];                                   // this row's scaled logits (log2 units)
   float mr[CPT];                                   // reference max per head, mirrored from smem
+  {   // zero the P buffer: its pad columns must read as zero
+    uint4* p = reinterpret_cast<uint4*>(r.smem + C::kP);
+    for (int k = tid; k < int(C::kPBytes / 16); k += 256) p[k] = make_uint4(0, 0, 0, 0);
+    named_barrier_softmax();
+  }
   TileWalk w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t pv_waited = -1;
@@ -674,6 +733,9 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
   }
 }
 
+// One CTA per SM.  The warps of a CTA are spread over the SM's four
+// sub-partitions of 16K registers each; with 11 warps three share one, which
+// caps a thread at 168 registers.
 template <int NP, int SK, int SV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
@@ -709,6 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(C::kOFull), 1);
     mbar_init(bar(C::kDone), 1);
     *r.abort = 0;
+    *reinterpret_cast<int*>(r.smem + C::kKIssued) = 0;
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
@@ -719,34 +782,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(r.sbase + C::kTmemSlot, kTmemCols);
     tmem_relinquish();
+    tc_fence_before();   // the block barriers of the schedule publish the slot
   }
   // Inputs may come from the kernel before this one on the stream (the append).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const WSched ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags,
-                                                     reinterpret_cast<int64_t*>(r.smem + C::kSched), kSegUnits);
-  const Sched& sc = ws.s;
-  r.seq0 = sc.seq;
-  r.lens_s = reinterpret_cast<const int*>(r.smem + C::kLens);
-  if (threadIdx.x < kLensCache && sc.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them
-    reinterpret_cast<int*>(r.smem + C::kLens)[threadIdx.x] =
-        clamp_len(__ldg(a.lens + sc.seq + threadIdx.x), a.m_max, nullptr, false);
-  if (threadIdx.x == 0) *reinterpret_cast<int*>(r.smem + C::kKIssued) = 0;
-  __syncthreads();
-  if (warp >= 2) {   // zero the P buffer (it held the schedule scratch): pad columns stay zero
-    uint4* p = reinterpret_cast<uint4*>(r.smem + C::kP);
-    for (int k = threadIdx.x - 64; k < int(C::kPBytes / 16); k += 256) p[k] = make_uint4(0, 0, 0, 0);
+  int* lens_tab = reinterpret_cast<int*>(r.smem + C::kLens);
+  r.lens_s = lens_tab;
+  int64_t* sched_red = reinterpret_cast<int64_t*>(r.smem + C::kSched);
+  WSched ws;
+  if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits)) {
+    ws = make_schedule_small<kThreads>(
+        a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab,
+        [&](int seq, int head, int k0, int own, int len, int nb) {
+          return pre_issue<NP, SK, SV>(a, r, &tm_k, &tm_v, &tm_q, seq, head, k0, own, len, nb);
+        });
+    r.seq0 = 0;
+  } else {
+    ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, sched_red,
+                                          kSegUnits);
+    r.seq0 = ws.s.seq;
+    if (threadIdx.x < kLensCache && ws.s.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them
+      lens_tab[threadIdx.x] = clamp_len(__ldg(a.lens + ws.s.seq + threadIdx.x), a.m_max, nullptr, false);
+    __syncthreads();
   }
-  tc_fence_before();
-  __syncthreads();
+  const Sched& sc = ws.s;
   tc_fence_after();
   r.tmem = *reinterpret_cast<volatile uint32_t*>(r.smem + C::kTmemSlot);
 
   if (sc.t_begin < sc.t_end) {
     if (warp == 0) {
       if (lane == 0) producer<NP, SK, SV, true>(a, ws, r, &tm_k, &tm_q);
-      else if (lane == 1) producer<NP, SK, SV, false>(a, ws, r, &tm_v, &tm_q);
     } else if (warp == 1) {
       if (lane == 0) mma_issuer<NP, SK, SV>(a, ws, r);
+    } else if (warp == kVWarp) {
+      // V loads from a warp of their own: sharing one with the K loads would
+      // serialise the two threads' waits
+      if (lane == 0) producer<NP, SK, SV, false>(a, ws, r, &tm_v, &tm_q);
     } else {
       softmax_epilogue<NP, SK, SV>(a, ws, r, warp, lane);
     }

@@ -244,3 +244,23 @@ def test_mixed_and_empty_lengths_many_ctas(path):
         ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, 1, wl.scale)
         assert_close(o, ref, "bf16", f"{path} ctas={ctas}")
         assert (o[lens == 0] == 0).all()
+
+
+@pytest.mark.parametrize("b", [352, 353, 700])
+def test_tensor_core_path_large_batches(b):
+    """Batches on both sides of the one-sequence-per-thread schedule (one
+    tensor-core CTA has 352 threads): every tile is owned by exactly one CTA
+    and zero-length sequences give zero rows."""
+    wl = small("bf16", b, 8, 1, 128, 300, 1, 1)
+    if not tc_available(wl):
+        pytest.skip("tensor-core path not built")
+    rng = np.random.default_rng(b)
+    lens = rng.integers(0, 301, size=b).astype(np.int32)
+    lens[rng.integers(0, b, size=b // 10)] = 0
+    inp = host_inputs(wl, seed=b, nan_tail=True, lens=np.maximum(lens, 1))
+    for ctas in (0, 37):
+        o = host64(binding.decode(dev(inp["q"], "bf16"), dev(inp["k"], "bf16"), dev(inp["v"], "bf16"),
+                                  torch.from_numpy(lens).cuda(), wl.scale, path="tcgen05", num_ctas=ctas))
+        ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, 1, wl.scale)
+        assert_close(o, ref, "bf16", f"b={b} ctas={ctas}")
+        assert (o[lens == 0] == 0).all()
