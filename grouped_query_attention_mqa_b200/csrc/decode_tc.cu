@@ -508,60 +508,32 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
   } pend;
   pend.on = false;
 
-  // Write a finished segment: O^T from tensor memory times 1/l, staged through
-  // the (idle) P buffer as [head][column] and stored with 16-byte copies; then
-  // the pad columns of P are zeroed again and the O buffer is released.
+  // Write a finished segment: O^T from tensor memory times 1/l.  Thread `row`
+  // holds output column `row` of its CPT heads, so for each head the 32 lanes
+  // of a warp store 32 consecutive columns (128 bytes of fp32 partial, 64 of
+  // bf16 output) straight from registers; then the O buffer is released.
   auto epilogue = [&](const Pending& e) {
     const int pb = e.sidx & 1;
-    unsigned char* stage = r.smem + C::kP;
-    constexpr int kPass = 32;                          // heads per fp32 pass (16 KB)
-    const int passes = e.whole ? 1 : (hq + kPass - 1) / kPass;
     const int64_t slot = partial_slot(blockIdx.x, e.seg);
-    float v[CPT], li[CPT];
+    float v[CPT];
     tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
+    if (e.whole) {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) +
+                           (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * kD + row;
 #pragma unroll
-    for (int k = 0; k < CPT; ++k) li[k] = linv[pb * NP + col0 + k];
+      for (int k = 0; k < CPT; ++k)
+        if (col0 + k < hq) dst[k * kD] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+    } else {
+      float* dst = a.ws.part_o + (slot * hq + col0) * kD + row;
 #pragma unroll
-    for (int k = 0; k < CPT; ++k) v[k] *= li[k];
-    for (int ps = 0; ps < passes; ++ps) {
-      const int c0 = e.whole ? 0 : ps * kPass;
-      const int nc = e.whole ? hq : min(kPass, hq - c0);
-      if (e.whole) {
-        __nv_bfloat16* st16 = reinterpret_cast<__nv_bfloat16*>(stage) + row;
-#pragma unroll
-        for (int k = 0; k < CPT; ++k)
-          if (col0 + k < hq) st16[(col0 + k) * kD] = __float2bfloat16_rn(v[k]);
-      } else {
-        float* st32 = reinterpret_cast<float*>(stage) + row;
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-          const int col = col0 + k - c0;
-          if (col >= 0 && col < nc) st32[col * kD] = v[k];
-        }
-      }
-      named_barrier_softmax();
-      const int esz = e.whole ? 2 : 4;
-      const int chunks = nc * kD * esz / 16;
-      uint4* dst = e.whole ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
-                                                      (int64_t(e.seq) * a.h + int64_t(e.head) * hq) * kD)
-                           : reinterpret_cast<uint4*>(a.ws.part_o + (slot * hq + c0) * kD);
-      const uint4* src = reinterpret_cast<const uint4*>(stage);
-      for (int k = tid; k < chunks; k += 256) dst[k] = src[k];
-      named_barrier_softmax();
+      for (int k = 0; k < CPT; ++k)
+        if (col0 + k < hq) dst[k * kD] = v[k] * linv[pb * NP + col0 + k];
     }
     if (warp == 2) {
       if (!e.whole)
         for (int col = lane; col < hq; col += 32) a.ws.part_lse[slot * hq + col] = lse2[pb * NP + col];
       if (e.owns_first && lane == 0)
         a.ws.seg_info[e.seg] = make_int2(blockIdx.x, cta_of_unit(e.seg_last_unit, ws.wtotal, sc.active));
-    }
-    if constexpr (NP < 64) {   // the staging overwrote the zero pad columns of P
-      if (grp == 1) {
-        unsigned char* prow0 = r.smem + C::kP + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-        for (int c8 = NP / 8; c8 < 8; ++c8)
-          *reinterpret_cast<uint4*>(prow0 + ((c8 ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
-      }
     }
     tc_fence_before();
     mbar_arrive(bar(C::kOFree + pb));
