@@ -64,7 +64,7 @@ constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
-constexpr int kSegUnits = 6;                 // cost of entering a segment, in quarter tiles (partition weight)
+constexpr int kSegUnits = 2;                 // cost of entering a segment, in quarter tiles (partition weight)
 constexpr int kLensCache = kThreads;         // clamped lengths kept in shared memory (all of them when b <= kThreads)
 constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O double buffer at [128, 256)
 constexpr uint32_t kOCol = 128;
