@@ -21,9 +21,6 @@ constexpr int kMergeThreads = 128;
 // issued by many threads at once instead of walked serially.
 template <typename T>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a, int heads_per_cta) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // The next step's decode may launch and set up while the merge runs.
-  asm volatile("griddepcontrol.launch_dependents;");
   const int hq = a.hq, D = a.d;
   const int chunks = (hq + heads_per_cta - 1) / heads_per_cta;
   const int64_t s = blockIdx.x / chunks;
@@ -31,10 +28,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
   const int tph = D / 4;                                    // threads per head
   const int i = hc * heads_per_cta + int(threadIdx.x) / tph;
   const int c4 = (int(threadIdx.x) % tph) * 4;
-  if (threadIdx.x >= heads_per_cta * tph || i >= hq) return;
+  const bool active = threadIdx.x < heads_per_cta * tph && i < hq;
   const int seq = int(s / a.g), head = int(s - int64_t(seq) * a.g);
+  // lens is an input of the call, never written by the decode kernel this
+  // merge follows, so it is read before waiting for that kernel.
+  const int len = active ? clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false) : 0;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The next step's decode may launch and set up while the merge runs.
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (!active) return;
   T* O = static_cast<T*>(a.o) + (int64_t(seq) * a.h + int64_t(head) * hq + i) * D + c4;
-  const int len = clamp_len(__ldg(a.lens + seq), a.m_max, nullptr, false);
   if (len == 0) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) O[k] = from_f32<T>(0.f);
@@ -42,18 +45,47 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
   }
   const int2 info = a.ws.seg_info[s];
   if (info.x == info.y) return;
-  float m = -INFINITY, wsum = 0.f;
+  // The loads of the first kParts partials go out together (one L2 round
+  // trip), then they are combined; a segment split more ways takes the rest
+  // one by one.
+  constexpr int kParts = 4;
+  const int nparts = info.y - info.x + 1;
+  float lse[kParts];
+  float4 v[kParts];
+#pragma unroll
+  for (int k = 0; k < kParts; ++k) {
+    lse[k] = -INFINITY;
+    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (k < nparts) {
+      const int64_t slot = partial_slot(info.x + k, s);
+      lse[k] = __ldcg(a.ws.part_lse + slot * hq + i);
+      v[k] = __ldcg(reinterpret_cast<const float4*>(a.ws.part_o + (slot * hq + i) * D + c4));
+    }
+  }
+  float m = lse[0];
+#pragma unroll
+  for (int k = 1; k < kParts; ++k) m = fmaxf(m, lse[k]);
+  float wsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k = info.x; k <= info.y; ++k) {
+#pragma unroll
+  for (int k = 0; k < kParts; ++k) {
+    const float w = exp2f(lse[k] - m);   // 0 for the absent parts (lse = -inf)
+    acc.x += w * v[k].x;
+    acc.y += w * v[k].y;
+    acc.z += w * v[k].z;
+    acc.w += w * v[k].w;
+    wsum += w;
+  }
+  for (int k = info.x + kParts; k <= info.y; ++k) {
     const int64_t slot = partial_slot(k, s);
-    const float lse = a.ws.part_lse[slot * hq + i];
-    const float4 v = *reinterpret_cast<const float4*>(a.ws.part_o + (slot * hq + i) * D + c4);
-    const float mn = fmaxf(m, lse);
-    const float cold = exp2f(m - mn), cnew = exp2f(lse - mn);
-    acc.x = acc.x * cold + cnew * v.x;
-    acc.y = acc.y * cold + cnew * v.y;
-    acc.z = acc.z * cold + cnew * v.z;
-    acc.w = acc.w * cold + cnew * v.w;
+    const float l = __ldcg(a.ws.part_lse + slot * hq + i);
+    const float4 u = __ldcg(reinterpret_cast<const float4*>(a.ws.part_o + (slot * hq + i) * D + c4));
+    const float mn = fmaxf(m, l);
+    const float cold = exp2f(m - mn), cnew = exp2f(l - mn);
+    acc.x = acc.x * cold + cnew * u.x;
+    acc.y = acc.y * cold + cnew * u.y;
+    acc.z = acc.z * cold + cnew * u.z;
+    acc.w = acc.w * cold + cnew * u.w;
     wsum = wsum * cold + cnew;
     m = mn;
   }
