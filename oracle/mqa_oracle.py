@@ -14,8 +14,10 @@ Sources (web pages on Multi-Query Attention; cited by title and section):
   einsums: logits = einsum("bhk,bmk->bhm", q, K); weights = softmax(logits);
   o = einsum("bhm,bmv->bhv", weights, V); the per-head form has K/V [b,h,m,k].
 * [kuangjux notes] "Fast Transformer Decoding: One Write-Head is All You Need"
-  (study notes), §1 (the scaled, masked softmax O = softmax(QKᵀ/√d_h + M)V) and
-  §4 (MQA drops only the head axis of K/V; worked example with two keys).
+  (study notes), §1 (the scaled, masked softmax O = softmax(QKᵀ/√d_h + M)V),
+  §4 (MQA drops only the head axis of K/V; worked example with two keys), §6.1
+  (the decoder's local attention: the current position and the 31 before it)
+  and §6.4 (local attention and MQA combined).
 * [oscine blog] "GQA、MQA、MLA：当「多头」变成推理账单上最贵的一项", section
   "第三站: GQA" (H query heads split into G groups, one K/V head per group;
   GQA-1 is MQA, GQA-H is MHA).
@@ -31,6 +33,10 @@ notes of the repository):
 * Grouping: query head i reads K/V head j(i) = i // (h // g), i.e. contiguous
   groups; h must be a multiple of g.
 * lens[b] == 0: the output row is 0 and lse is -inf (the pages do not define it).
+* Local window: the notes name a window of the current position plus the 31
+  before it, with no formula.  With ``window`` = w > 0, position t of sequence
+  b is attended iff lens[b] - w <= t < lens[b] (the newest w rows; w = 32 is the
+  notes' window); w = 0 means no window.
 
 Parity pins for every function live in ``tests/test_oracle.py``; none is
 unpinned.
@@ -78,7 +84,7 @@ def dot_product_attention(q, K, V, scale=1.0):
     return np.array(y, dtype=np.float64), np.array(weights, dtype=np.float64)
 
 
-def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
+def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False, window=0):
     """One decode step of MQA / GQA / MHA attention, in float64.
 
     Shapes: q [b, h, d_k]; k_cache [b, m_max, g, d_k]; v_cache [b, m_max, g, d_v];
@@ -92,6 +98,8 @@ def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
         w = softmax over the L valid positions      (§3 softmax; [kuangjux notes] §1)
         o = w V_j                                   (§3 weighted-V einsum)
     g = 1 is MQA, g = h is MHA, 1 < g < h is GQA ([oscine blog] "第三站: GQA").
+    With ``window`` = w > 0 only positions L-w <= t < L take part (local
+    attention, [kuangjux notes] §6.1 and §6.4); the weights of the others are 0.
     Inputs are used at whatever precision they hold (the tests hand in values
     already rounded to the kernel's input type) and widened to float64 here.
     """
@@ -105,6 +113,9 @@ def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
     if g_cache != g or h % g != 0:
         raise ValueError("k_cache must have g heads and h must be a multiple of g")
     hq = h // g
+    window = int(window)
+    if window < 0:
+        raise ValueError("window must be >= 0")
     o = np.zeros((b, h, d_v), dtype=np.float64)
     lse = np.full((b, h), -np.inf, dtype=np.float64)
     weights = [] if return_weights else None
@@ -117,10 +128,11 @@ def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
             if return_weights:
                 weights.append(w_b)
             continue
+        L0 = max(0, L - window) if window > 0 else 0                        # first attended row
         for j in range(g):
             Qj = q[bi, j * hq:(j + 1) * hq, :].astype(np.float64)          # [hq, d_k]
-            Kj = k_cache[bi, :L, j, :].astype(np.float64)                   # [L, d_k]
-            Vj = v_cache[bi, :L, j, :].astype(np.float64)                   # [L, d_v]
+            Kj = k_cache[bi, L0:L, j, :].astype(np.float64)                 # [L-L0, d_k]
+            Vj = v_cache[bi, L0:L, j, :].astype(np.float64)                 # [L-L0, d_v]
             S = scale * (Qj @ Kj.T)                                         # [hq, L]
             mu = S.max(axis=1, keepdims=True)
             E = np.exp(S - mu)
@@ -128,7 +140,7 @@ def oracle_decode(q, k_cache, v_cache, lens, g, scale, return_weights=False):
             W = E / denom
             o[bi, j * hq:(j + 1) * hq, :] = W @ Vj
             lse[bi, j * hq:(j + 1) * hq] = (mu + np.log(denom))[:, 0]
-            w_b[j * hq:(j + 1) * hq, :] = W
+            w_b[j * hq:(j + 1) * hq, L0:] = W
         if return_weights:
             weights.append(w_b)
     if return_weights:
@@ -156,10 +168,11 @@ def oracle_kv_append(k_cache, v_cache, k_new, v_new, pos):
     return k_out, v_out
 
 
-def oracle_decode_step(q, k_cache, v_cache, k_new, v_new, lens_before, g, scale):
+def oracle_decode_step(q, k_cache, v_cache, k_new, v_new, lens_before, g, scale, window=0):
     """One whole incremental step in the order of [velog review] §3: append the
-    new K/V at row lens_before[b], then attend over lens_before[b] + 1 rows."""
+    new K/V at row lens_before[b], then attend over lens_before[b] + 1 rows (the
+    newest ``window`` of them when window > 0)."""
     k2, v2 = oracle_kv_append(k_cache, v_cache, k_new, v_new, lens_before)
     lens_after = np.asarray(lens_before).astype(np.int64) + 1
-    o, lse = oracle_decode(q, k2, v2, lens_after, g, scale)
+    o, lse = oracle_decode(q, k2, v2, lens_after, g, scale, window=window)
     return o, lse, k2, v2

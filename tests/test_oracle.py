@@ -329,3 +329,86 @@ def test_mha_over_mqa_cache_bytes_is_h():
     a = kv_cache_bytes(mha.b, mha.m_max, mha.g, mha.d_k, mha.d_v, mha.elem_bytes)
     c = kv_cache_bytes(mqa.b, mqa.m_max, mqa.g, mqa.d_k, mqa.d_v, mqa.elem_bytes)
     assert a == 32 * c and a == 4 * 2**30
+
+
+# ------------------------------------------------------------ local window
+
+def test_window_one_returns_the_newest_row_of_v(golden):
+    """Study notes §6.1/§6.4 local attention with a window of one position: the
+    softmax has one term, so every head returns V at row L-1 and lse is that
+    row's logit.  On the two-key example the window keeps only k2/v2."""
+    g = golden("worked_example_two_keys.txt")
+    q, K, V = _two_key_problem(g)
+    o, lse, w = oracle_decode(q, K, V, [2], g=1, scale=1.0, return_weights=True, window=1)
+    np.testing.assert_array_equal(w[0], [[0.0, 1.0], [0.0, 1.0]])
+    np.testing.assert_array_equal(o[0], [g["v2"], g["v2"]])
+    np.testing.assert_allclose(lse[0], [float(np.dot(g["q1"], g["k2"])), float(np.dot(g["q2"], g["k2"]))],
+                               rtol=0, atol=1e-15)
+
+
+def test_window_covering_the_cache_is_full_attention(golden):
+    """A window at least as long as the sequence leaves every row in."""
+    g = golden("worked_example_two_keys.txt")
+    q, K, V = _two_key_problem(g)
+    for window in (2, 3, 100):
+        _, _, w = oracle_decode(q, K, V, [2], g=1, scale=1.0, return_weights=True, window=window)
+        np.testing.assert_allclose(w[0][0], g["scale_1.head1"], rtol=0, atol=1e-15)
+        np.testing.assert_allclose(w[0][1], g["scale_1.head2"], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("window", [1, 3, 5, 32])
+def test_window_is_brute_force_on_the_newest_rows(window):
+    """With window w the result is DotProductAttention over rows L-w .. L-1 only,
+    computed by the per-query brute force on that slice; rows before the
+    window hold NaN and must not be read."""
+    rng = np.random.default_rng(40 + window)
+    b, h, g, m, d = 3, 4, 2, 40, 5
+    q = _rand(rng, b, h, d)
+    K = _rand(rng, b, m, g, d)
+    V = _rand(rng, b, m, g, d)
+    lens = [40, 7, 2]
+    Kn, Vn = K.copy(), V.copy()
+    for bi, L in enumerate(lens):
+        lo = max(0, L - window)
+        Kn[bi, :lo] = np.nan
+        Vn[bi, :lo] = np.nan
+        Kn[bi, L:] = np.nan
+        Vn[bi, L:] = np.nan
+    o, lse, w = oracle_decode(q, Kn, Vn, lens, g=g, scale=0.7, return_weights=True, window=window)
+    assert np.isfinite(o).all()
+    for bi, L in enumerate(lens):
+        lo = max(0, L - window)
+        assert np.count_nonzero(w[bi]) == h * (L - lo)
+        for i in range(h):
+            j = i // (h // g)
+            y, wi = dot_product_attention(q[bi, i], K[bi, lo:L, j], V[bi, lo:L, j], scale=0.7)
+            np.testing.assert_allclose(o[bi, i], y, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(w[bi][i, lo:], wi, rtol=0, atol=1e-15)
+
+
+def test_notes_window_is_current_plus_31_previous():
+    """Study notes §6.1: the decoder window is the current position and the 31
+    before it, i.e. window=32 attends rows L-32 .. L-1 (exactly 32 of them)."""
+    rng = np.random.default_rng(41)
+    L = 100
+    q = _rand(rng, 1, 2, 4)
+    K = _rand(rng, 1, L, 1, 4)
+    V = _rand(rng, 1, L, 1, 4)
+    _, _, w = oracle_decode(q, K, V, [L], g=1, scale=1.0, return_weights=True, window=32)
+    nz = np.nonzero(w[0][0])[0]
+    assert nz.min() == L - 32 and nz.max() == L - 1 and len(nz) == 32
+
+
+def test_step_with_window_attends_the_appended_row():
+    """The appended row is the newest one, so it is inside any window: with
+    window=1 the step returns the new V row for every head."""
+    rng = np.random.default_rng(42)
+    b, h, g, m, d = 2, 4, 2, 9, 3
+    q = _rand(rng, b, h, d)
+    K = _rand(rng, b, m, g, d)
+    V = _rand(rng, b, m, g, d)
+    kn, vn = _rand(rng, b, g, d), _rand(rng, b, g, d)
+    o, _, _, _ = oracle_decode_step(q, K, V, kn, vn, [3, 8], g=g, scale=1.0, window=1)
+    for bi in range(b):
+        for i in range(h):
+            np.testing.assert_array_equal(o[bi, i], vn[bi, i // (h // g)])
