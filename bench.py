@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
     p.add_argument("--num-ctas", type=int, default=0)
+    p.add_argument("--window", type=int, default=0, help="local attention: attend to the newest W rows (0 = all)")
     p.add_argument("--e2e-steps", type=int, default=3000)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -83,7 +84,7 @@ def blas_threads():
         return 1
 
 
-def time_oracle(wl, seconds, n_seq=16):
+def time_oracle(wl, seconds, n_seq=16, window=0):
     """Oracle steps (append, then attend) over sampled sequences until about
     `seconds` of CPU time has passed.  Returns (tokens/s, sequences, seconds)."""
     from oracle import oracle_decode_step   # test infrastructure: only this leg of the bench runs it
@@ -96,15 +97,15 @@ def time_oracle(wl, seconds, n_seq=16):
             cache_k = np.concatenate([s["k"], np.zeros((1, 1, wl.g, wl.d_k), np.float32)], axis=1)
             cache_v = np.concatenate([s["v"], np.zeros((1, 1, wl.g, wl.d_v), np.float32)], axis=1)
             oracle_decode_step(s["q"], cache_k, cache_v, s["k_new"], s["v_new"], np.array([s["L"] - 1]), wl.g,
-                               wl.scale)
+                               wl.scale, window=window)
             done += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             return done / el, done, el
 
 
-def cpu_baseline_obj(wl, seconds):
-    v, n, el = time_oracle(wl, seconds)
+def cpu_baseline_obj(wl, seconds, window=0):
+    v, n, el = time_oracle(wl, seconds, window=window)
     return {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} sequence-steps of {wl.name} (first 16 sequences of seed {SEED}, valid rows only), "
                       f"NumPy float64 append+attend, {el:.1f} s"}
@@ -117,10 +118,10 @@ def run_reference(args):
     wl = WORKLOADS[args.workload]
     per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        time_oracle(wl, 0.0, n_seq=2)
+        time_oracle(wl, 0.0, n_seq=2, window=args.window)
     rates, total_n, total_t = [], 0, 0.0
     for _ in range(args.steps):
-        v, n, el = time_oracle(wl, per_step)
+        v, n, el = time_oracle(wl, per_step, window=args.window)
         rates.append(v)
         total_n += n
         total_t += el
@@ -295,6 +296,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     # one pre-marshalled fused step (append at row lens-1, then decode) per cache copy
     steps = [binding.DecodePlan(inp["q"], inp["k"][c], inp["v"][c], lens, wl.scale, out=out, workspace=ws,
+                                window=args.window,
                                 path=path, num_ctas=args.num_ctas, k_new=inp["k_new"], v_new=inp["v_new"])
              for c in range(copies)]
 
@@ -364,6 +366,7 @@ def run_ours(args):
                   o_h=torch.empty(out.shape, dtype=out.dtype).pin_memory(),
                   in_ready=torch.cuda.Event(), computed=torch.cuda.Event(), out_done=torch.cuda.Event())
         sl["plans"] = [binding.DecodePlan(sl["q"], inp["k"][c], inp["v"][c], sl["lens"], wl.scale, out=sl["out"],
+                                          window=args.window,
                                           workspace=ws, path=path, num_ctas=args.num_ctas, stream=cap,
                                           k_new=sl["kn"], v_new=sl["vn"]) for c in range(copies)]
         slots.append(sl)
@@ -421,7 +424,7 @@ def run_ours(args):
     e2e_ms = reduce_over_ranks([s2.elapsed_time(e2)], "cuda")[0]
     e2e_value = job_value(world, b, E, e2e_ms)
 
-    alg_bytes = decode_algorithmic_bytes(wl, lens_np) + append_algorithmic_bytes(wl)
+    alg_bytes = decode_algorithmic_bytes(wl, lens_np, args.window) + append_algorithmic_bytes(wl)
     peak, peak_kind = peaks()
     achieved = alg_bytes / (dec_avg_ms / 1e3) / 1e9
     kernel = "decode_tc_kernel" if path == "tcgen05" else "decode_simt_kernel"
@@ -431,18 +434,20 @@ def run_ours(args):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline_obj(wl, args.cpu_seconds)
+            cpu = cpu_baseline_obj(wl, args.cpu_seconds, args.window)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "b": b, "h": h, "g": g, "d": d, "m_max": wl.m_max,
                        "lens": f"U[{wl.len_lo},{wl.len_hi}] (seed {SEED}+rank), mean {float(lens_np.mean()):.0f}",
-                       "step": "mqa_decode_append: new K/V row written at lens-1, then attention over lens rows",
+                       "step": "mqa_decode_append: new K/V row written at lens-1, then attention over lens rows"
+                               + (f" (the newest {args.window}: local window)" if args.window else ""),
                        "path": path,
                        "l2": f"{copies} rotating K/V cache copies ({copies * cache_bytes / 2**20:.0f} MiB) so each "
                              f"step's rows were evicted by >= 2 other steps' reads",
-                       "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)"},
+                       "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)",
+                       **({"window": args.window} if args.window else {})},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": f"one step = mqa_decode_append call ({kernel} + merge_kernel), average over "

@@ -27,7 +27,7 @@ _c_int, _c_size, _c_ptr, _c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void
 
 
 class DecodeOptions(ctypes.Structure):
-    _fields_ = [("path", _c_int), ("num_ctas", _c_int)]
+    _fields_ = [("path", _c_int), ("num_ctas", _c_int), ("window", _c_int)]
 
 
 SIGNATURES = {
@@ -148,9 +148,10 @@ _ws = _WsCache()
 
 
 def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_flags=None, path="auto",
-           num_ctas=0, stream=None):
+           num_ctas=0, stream=None, window=0):
     """o [b,h,d_v] = softmax over rows t < lens[b] of scale·q·K, times V
-    (mqa_decode_ex).  ``workspace`` defaults to a torch-allocated buffer of
+    (mqa_decode_ex); with ``window`` > 0 over the newest ``window`` rows only.
+    ``workspace`` defaults to a torch-allocated buffer of
     mqa_decode_workspace_size bytes, kept for reuse."""
     import torch
     _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags)
@@ -175,7 +176,7 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
             ws = new_workspace(b, h, g, d_v, device=q.device)
             _ws.tensor = ws
         workspace = ws
-    opts = DecodeOptions(PATHS[path], int(num_ctas))
+    opts = DecodeOptions(PATHS[path], int(num_ctas), int(window))
     st = lib().mqa_decode_ex(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), b, h, g, m_max, d_k, d_v,
                              float(scale), dt, _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _ptr(status_flags), ctypes.byref(opts), _stream_handle(stream))
@@ -185,11 +186,12 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
 
 
 def decode_append(q, k_cache, v_cache, k_new, v_new, lens, scale, out=None, workspace=None, status_flags=None,
-                  path="auto", num_ctas=0, stream=None):
+                  path="auto", num_ctas=0, stream=None, window=0):
     """One incremental step (mqa_decode_append): write k_new/v_new [b,g,d] at
-    row lens[b]-1 of the caches, then attend over lens[b] rows.  Returns o."""
+    row lens[b]-1 of the caches, then attend over lens[b] rows (the newest
+    ``window`` of them when window > 0).  Returns o."""
     plan = DecodePlan(q, k_cache, v_cache, lens, scale, out=out, workspace=workspace, status_flags=status_flags,
-                      path=path, num_ctas=num_ctas, stream=stream, k_new=k_new, v_new=v_new)
+                      path=path, num_ctas=num_ctas, stream=stream, k_new=k_new, v_new=v_new, window=window)
     return plan.run()
 
 
@@ -220,7 +222,7 @@ class DecodePlan:
     that writes ``self.out``."""
 
     def __init__(self, q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_flags=None, path="auto",
-                 num_ctas=0, stream=None, k_new=None, v_new=None):
+                 num_ctas=0, stream=None, k_new=None, v_new=None, window=0):
         import torch
         _check_cuda(q, k_cache, v_cache, lens, out, workspace, status_flags, k_new, v_new)
         b, h, d_k = q.shape
@@ -239,7 +241,7 @@ class DecodePlan:
         if workspace is None:
             workspace = new_workspace(b, h, g, d_v, device=q.device)
         self.out = out
-        self._opts = DecodeOptions(PATHS[path], int(num_ctas))
+        self._opts = DecodeOptions(PATHS[path], int(num_ctas), int(window))
         self._keep = (q, k_cache, v_cache, lens, out, workspace, status_flags, k_new, v_new)
         common = (ctypes.c_float(scale), _dtype_code(q), _ptr(workspace), workspace.numel() * workspace.element_size(),
                   _ptr(status_flags), ctypes.byref(self._opts), _stream_handle(stream))

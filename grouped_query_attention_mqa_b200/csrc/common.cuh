@@ -106,6 +106,12 @@ struct Sched {
 
 __device__ __forceinline__ int tiles_of(int len, int tile) { return (len + tile - 1) / tile; }
 
+// Rows of a sequence of length len that a decode attends to: all of them, or
+// with a local window w > 0 the newest min(len, w) ("Fast Transformer
+// Decoding" study notes §6.1, §6.4).  Partitions count tiles of the span;
+// tile k of a segment starts at cache row (len - span) + k * tile.
+__device__ __forceinline__ int span_of(int len, int window) { return window > 0 && len > window ? window : len; }
+
 __device__ __forceinline__ int64_t range_start(int64_t c, int64_t total, int active) {
   return (c * total) / active;
 }
@@ -122,7 +128,7 @@ __device__ __forceinline__ int cta_of_tile(int64_t t, int64_t total, int active)
 // Cost: O(b / NT) loads per thread and three block barriers.
 // `red` needs NT/32 + 2 int64 of shared memory.
 template <int NT>
-__device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile,
+__device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, int m_max, int window, int tile,
                                int grid, int cta, int32_t* flags, int64_t* red) {
   static_assert(NT % 32 == 0, "whole warps");
   const int per = (b + NT - 1) / NT;
@@ -130,7 +136,7 @@ __device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, i
   const int s1 = min(b, s0 + per);
   int64_t mine = 0;
   for (int s = s0; s < s1; ++s)
-    mine += int64_t(g) * tiles_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), tile);
+    mine += int64_t(g) * tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), window), tile);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t x = mine;
 #pragma unroll
@@ -163,7 +169,7 @@ __device__ Sched make_schedule(const int32_t* __restrict__ lens, int b, int g, i
   if (sc.t_begin >= excl && sc.t_begin < excl + mine) {
     int64_t base = excl;
     for (int s = s0; s < s1; ++s) {
-      int64_t n = int64_t(g) * tiles_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), tile);
+      int64_t n = int64_t(g) * tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), window), tile);
       if (sc.t_begin < base + n) {
         out[0] = s;
         out[1] = base;
@@ -203,15 +209,15 @@ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t wtotal, int active
 }
 
 template <int NT>
-__device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile,
-                                         int grid, int cta, int32_t* flags, int64_t* red, int xw) {
+__device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b, int g, int m_max, int window,
+                                         int tile, int grid, int cta, int32_t* flags, int64_t* red, int xw) {
   static_assert(NT % 32 == 0, "whole warps");
   const int per = (b + NT - 1) / NT;
   const int s0 = min(b, int(threadIdx.x) * per);
   const int s1 = min(b, s0 + per);
   int64_t my_t = 0, my_u = 0;
   for (int s = s0; s < s1; ++s) {
-    const int nb = tiles_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), tile);
+    const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), window), tile);
     my_t += int64_t(g) * nb;
     my_u += seq_units(nb, g, xw);
   }
@@ -266,7 +272,7 @@ __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b
     if (!(u >= excl_u && u < excl_u + my_u)) return;
     int64_t tb = excl_t, ub = excl_u;
     for (int s = s0; s < s1; ++s) {
-      const int nb = tiles_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), tile);
+      const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), window), tile);
       const int64_t su = seq_units(nb, g, xw);
       if (u < ub + su) {
         const int64_t seglen = xw + 4 * int64_t(nb);
@@ -314,8 +320,8 @@ __device__ __forceinline__ bool small_schedule_fits(int b, int g, int m_max, int
 }
 
 template <int NT, typename OnFirst>
-__device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, int g, int m_max, int tile, int grid,
-                                      int cta, int32_t* flags, int64_t* red, int xw, int* lens_tab,
+__device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, int g, int m_max, int window, int tile,
+                                      int grid, int cta, int32_t* flags, int64_t* red, int xw, int* lens_tab,
                                       OnFirst&& on_first) {
   static_assert(NT % 32 == 0, "whole warps");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -324,7 +330,7 @@ __device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, i
     len = clamp_len(__ldg(lens + tid), m_max, flags, cta == 0);
     lens_tab[tid] = len;
   }
-  const int nb = tiles_of(len, tile);
+  const int nb = tiles_of(span_of(len, window), tile);
   const int my_t = g * nb;
   const int my_u = nb > 0 ? g * (xw + 4 * nb) : 0;
   uint64_t x = (uint64_t(uint32_t(my_t)) << 32) | uint32_t(my_u);
@@ -401,26 +407,29 @@ struct Cursor {
   int64_t base;     // first tile of that sequence
   int nb;           // tiles per segment of that sequence
   int len;          // clamped length of that sequence
+  int lo;           // first attended row (len - span)
 };
 
-__device__ __forceinline__ Cursor cursor_at(const int32_t* __restrict__ lens, int m_max, int tile, int seq,
-                                            int64_t base) {
+__device__ __forceinline__ Cursor cursor_at(const int32_t* __restrict__ lens, int m_max, int window, int tile,
+                                            int seq, int64_t base) {
   Cursor cu;
   cu.seq = seq;
   cu.base = base;
   cu.len = clamp_len(__ldg(lens + seq), m_max, nullptr, false);
-  cu.nb = tiles_of(cu.len, tile);
+  cu.lo = cu.len - span_of(cu.len, window);
+  cu.nb = tiles_of(cu.len - cu.lo, tile);
   return cu;
 }
 
 // Advance the cursor until tile t lies in its sequence.
 __device__ __forceinline__ void cursor_seek(Cursor& cu, const int32_t* __restrict__ lens, int g, int m_max,
-                                            int tile, int64_t t) {
+                                            int window, int tile, int64_t t) {
   while (t >= cu.base + int64_t(g) * cu.nb) {
     cu.base += int64_t(g) * cu.nb;
     cu.seq += 1;
     cu.len = clamp_len(__ldg(lens + cu.seq), m_max, nullptr, false);
-    cu.nb = tiles_of(cu.len, tile);
+    cu.lo = cu.len - span_of(cu.len, window);
+    cu.nb = tiles_of(cu.len - cu.lo, tile);
   }
 }
 
@@ -438,7 +447,7 @@ __device__ __forceinline__ TileCoord tile_coord(const Cursor& cu, int g, int til
   tc.seq = cu.seq;
   tc.head = int(rel / cu.nb);
   tc.k = int(rel - int64_t(tc.head) * cu.nb);
-  tc.row0 = tc.k * tile;
+  tc.row0 = cu.lo + tc.k * tile;
   tc.rows = min(tile, cu.len - tc.row0);
   tc.seg = int64_t(cu.seq) * g + tc.head;
   tc.nb = cu.nb;
@@ -460,6 +469,7 @@ struct DecodeArgs {
   const int32_t* lens;
   int b, h, g, m_max, d;
   int hq;
+  int window;          // local attention: the newest `window` rows (0 = all rows)
   float scale;
   Workspace ws;
   int32_t* flags;

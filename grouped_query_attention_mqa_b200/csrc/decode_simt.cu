@@ -150,15 +150,15 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
 
   // Inputs may come from the kernel before this one on the stream (the append).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const Sched sc = make_schedule<kThreads>(a.lens, a.b, g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, red);
+  const Sched sc = make_schedule<kThreads>(a.lens, a.b, g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, red);
   if (sc.t_begin >= sc.t_end) {
     asm volatile("griddepcontrol.launch_dependents;");
     return;
   }
 
-  Cursor cur = cursor_at(a.lens, a.m_max, kTile, sc.seq, sc.seq_base);
+  Cursor cur = cursor_at(a.lens, a.m_max, a.window, kTile, sc.seq, sc.seq_base);
   Cursor nxt = cur;
-  cursor_seek(cur, a.lens, g, a.m_max, kTile, sc.t_begin);
+  cursor_seek(cur, a.lens, g, a.m_max, a.window, kTile, sc.t_begin);
   {
     const TileCoord t0 = tile_coord(cur, g, kTile, sc.t_begin);
     load_tile<T, D>(stage, stage + 2 * kStageBytes, K, V, t0, g, a.m_max, KN, VN);
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
 
   for (int64_t t = sc.t_begin; t < sc.t_end; ++t) {
     const int st = int((t - sc.t_begin) & 1);
-    cursor_seek(cur, a.lens, g, a.m_max, kTile, t);
+    cursor_seek(cur, a.lens, g, a.m_max, a.window, kTile, t);
     const TileCoord tc = tile_coord(cur, g, kTile, t);
 
     if (t == sc.t_begin || tc.k == 0) {   // a new segment starts: its queries, fresh state
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
       for (int r = 0; r < kMaxOutPairs; ++r) acc[r] = make_float2(0.f, 0.f);
     }
     if (t + 1 < sc.t_end) {
-      cursor_seek(nxt, a.lens, g, a.m_max, kTile, t + 1);
+      cursor_seek(nxt, a.lens, g, a.m_max, a.window, kTile, t + 1);
       const TileCoord tn = tile_coord(nxt, g, kTile, t + 1);
       load_tile<T, D>(stage + (st ^ 1) * kStageBytes, stage + (2 + (st ^ 1)) * kStageBytes, K, V, tn, g,
                       a.m_max, KN, VN);

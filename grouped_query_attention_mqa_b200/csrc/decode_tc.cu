@@ -195,6 +195,7 @@ struct TileWalk {
   int64_t base;              // first tile of the current sequence
   int64_t ubase;             // first partition unit of the current sequence
   int seq, head, k, nb, len;
+  int lo;                    // first attended row of the sequence (len - span)
   int sidx;                  // segment number within this CTA
   TileCoord tc;
   bool first, last;
@@ -203,18 +204,21 @@ struct TileWalk {
     seq = ws.s.seq;
     base = ws.s.seq_base;
     ubase = ws.seq_ubase;
-    len = seq_len(a, r, seq);
-    nb = tiles_of(len, kTile);
+    set_seq(a, r, seq);
     while (ws.s.t_begin >= base + int64_t(a.g) * nb) {   // the first tile may lie in a later sequence
       base += int64_t(a.g) * nb;
       ubase += seq_units(nb, a.g, kSegUnits);
-      ++seq;
-      len = seq_len(a, r, seq);
-      nb = tiles_of(len, kTile);
+      set_seq(a, r, seq + 1);
     }
     const int rel = int(ws.s.t_begin - base);   // < g * nb
     head = rel / nb;
     k = rel - head * nb - 1;                     // next() advances to the first tile
+  }
+  __device__ void set_seq(const DecodeArgs& a, const Roles& r, int s) {
+    seq = s;
+    len = seq_len(a, r, s);
+    lo = len - span_of(len, a.window);
+    nb = tiles_of(len - lo, kTile);
   }
   __device__ void next(const DecodeArgs& a, const Sched& sc) {
     ++t;
@@ -225,16 +229,14 @@ struct TileWalk {
         base += int64_t(a.g) * nb;
         ubase += seq_units(nb, a.g, kSegUnits);
         do {
-          ++seq;
-          len = seq_len(a, *rr, seq);
-          nb = tiles_of(len, kTile);
+          set_seq(a, *rr, seq + 1);
         } while (nb == 0);
       }
     }
     tc.seq = seq;
     tc.head = head;
     tc.k = k;
-    tc.row0 = k * kTile;
+    tc.row0 = lo + k * kTile;
     tc.rows = min(kTile, len - tc.row0);
     tc.seg = int64_t(seq) * a.g + head;
     tc.nb = nb;
@@ -288,7 +290,8 @@ __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap*
       append_new_row(a, true, seq, head, len);
       append_new_row(a, false, seq, head, len);
     }
-    const int row = seq * a.m_max + k * kTile;
+    const int row0 = len - span_of(len, a.window) + k * kTile;
+    const int row = seq * a.m_max + row0;
     const uint32_t kdst = r.sbase + C::kK + i * kTileBytes;
     mbar_expect_tx(bar(C::kKFull + i), kTileBytes);
     tma_load_3d(kdst, tm_k, bar(C::kKFull + i), 0, head, row, pol);
@@ -764,13 +767,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   WSched ws;
   if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits)) {
     ws = make_schedule_small<kThreads>(
-        a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab,
+        a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab,
         [&](int seq, int head, int k0, int own, int len, int nb) {
           return pre_issue<NP, SK, SV>(a, r, &tm_k, &tm_v, &tm_q, seq, head, k0, own, len, nb);
         });
     r.seq0 = 0;
   } else {
-    ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, kTile, a.grid, blockIdx.x, a.flags, sched_red,
+    ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red,
                                           kSegUnits);
     r.seq0 = ws.s.seq;
     if (threadIdx.x < kLensCache && ws.s.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them

@@ -76,7 +76,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
     return MQA_ERR_INVALID_ARG;
   const int path = opts ? opts->path : MQA_PATH_AUTO;
   if (path < MQA_PATH_AUTO || path > MQA_PATH_TCGEN05) return MQA_ERR_INVALID_ARG;
-  if (opts && (opts->num_ctas < 0 || opts->num_ctas > kMaxCtas)) return MQA_ERR_INVALID_ARG;
+  if (opts && (opts->num_ctas < 0 || opts->num_ctas > kMaxCtas || opts->window < 0)) return MQA_ERR_INVALID_ARG;
   if (b == 0) return MQA_OK;
   if (!o || !q || !k_cache || !v_cache || !lens || !workspace) return MQA_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return MQA_ERR_INVALID_ARG;
@@ -120,6 +120,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.m_max = m_max;
   a.d = d_k;
   a.hq = hq;
+  a.window = opts ? opts->window : 0;
   a.scale = scale;
   a.ws = carve_workspace(workspace, b, g, hq);
   a.flags = status_flags;

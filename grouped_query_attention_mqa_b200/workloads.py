@@ -201,10 +201,13 @@ def kv_cache_bytes(b: int, m: int, g: int, d_k: int, d_v: int, elem_bytes: int) 
     return b * m * g * (d_k + d_v) * elem_bytes
 
 
-def decode_algorithmic_bytes(wl: Workload, lens) -> int:
-    """Bytes one decode must move at minimum: every valid K and V row once,
-    q read once, o written once.  Masked rows and split partials not counted."""
+def decode_algorithmic_bytes(wl: Workload, lens, window: int = 0) -> int:
+    """Bytes one decode must move at minimum: every attended K and V row once
+    (the valid rows, or the newest ``window`` of them), q read once, o written
+    once.  Masked rows and split partials not counted."""
     lens = np.asarray(lens, dtype=np.int64)
+    if window > 0:
+        lens = np.minimum(lens, window)
     kv = int(lens.sum()) * wl.g * (wl.d_k + wl.d_v) * wl.elem_bytes
     qo = wl.b * wl.h * (wl.d_k + wl.d_v) * wl.elem_bytes
     return kv + qo

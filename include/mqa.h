@@ -81,6 +81,14 @@ typedef enum {
 typedef struct {
   int path;                  /* mqa_path_t                                     */
   int num_ctas;              /* persistent CTAs; 0 = SM count x resident CTAs  */
+  int window;                /* local attention: attend only to the newest
+                                `window` valid rows of each sequence, rows
+                                [max(0, lens[b] - window), lens[b]); 0 = all
+                                rows.  "Fast Transformer Decoding" study notes
+                                §6.1 (the decoder's window: the current
+                                position and the 31 before it, window = 32)
+                                and §6.4 (local attention combined with MQA).
+                                Must be >= 0.                                  */
 } mqa_decode_opts_t;
 
 /* Largest number of persistent CTAs a decode may use; sizes the workspace. */

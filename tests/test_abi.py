@@ -88,6 +88,8 @@ def test_decode_rejects_bad_arguments_without_launching(lib):
     assert _decode(lib, opts=ctypes.byref(opts)) == INV  # unknown path
     opts = binding.DecodeOptions(0, binding.MQA_MAX_CTAS + 1)
     assert _decode(lib, opts=ctypes.byref(opts)) == INV
+    opts = binding.DecodeOptions(0, 0, -1)               # negative local window
+    assert _decode(lib, opts=ctypes.byref(opts)) == INV
     opts = binding.DecodeOptions(1, 0)                   # SIMT cannot take h/g*d > 4096
     assert _decode(lib, h=64, opts=ctypes.byref(opts)) == UNS
     opts = binding.DecodeOptions(2, 0)                   # tensor cores need bf16
