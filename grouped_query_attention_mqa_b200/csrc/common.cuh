@@ -470,6 +470,8 @@ struct DecodeArgs {
   int b, h, g, m_max, d;
   int hq;
   int window;          // local attention: the newest `window` rows (0 = all rows)
+  int no_merge;        // no segment spans two tiles: the decode writes every output row
+                       // itself (zero rows for empty sequences) and no merge follows
   float scale;
   Workspace ws;
   int32_t* flags;
@@ -484,6 +486,8 @@ int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq);
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 int tc_ctas_per_sm(int hq);
+int tc_tile_rows();
+int simt_tile_rows();
 bool tc_supported(int d, int hq);
 
 }  // namespace mqa

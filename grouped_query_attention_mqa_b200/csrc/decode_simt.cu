@@ -151,6 +151,14 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   // Inputs may come from the kernel before this one on the stream (the append).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const Sched sc = make_schedule<kThreads>(a.lens, a.b, g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, red);
+  if (a.no_merge) {   // no merge follows: empty sequences get their zero rows here
+    for (int s = blockIdx.x; s < a.b; s += gridDim.x) {
+      if (clamp_len(__ldg(a.lens + s), a.m_max, nullptr, false) == 0) {
+        T* o = static_cast<T*>(a.o) + int64_t(s) * a.h * D;
+        for (int k = threadIdx.x; k < a.h * D; k += kThreads) o[k] = from_f32<T>(0.f);
+      }
+    }
+  }
   if (sc.t_begin >= sc.t_end) {
     asm volatile("griddepcontrol.launch_dependents;");
     return;
@@ -353,6 +361,8 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStrea
   }
   return cudaErrorInvalidValue;
 }
+
+int simt_tile_rows() { return kTile; }
 
 int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq) {
   if (dtype == MQA_BF16) {

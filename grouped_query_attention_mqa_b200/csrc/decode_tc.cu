@@ -783,6 +783,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Sched& sc = ws.s;
   tc_fence_after();
   r.tmem = *reinterpret_cast<volatile uint32_t*>(r.smem + C::kTmemSlot);
+  if (a.no_merge && warp >= 2 && warp < kVWarp) {   // no merge follows: empty sequences get their zero rows here
+    for (int s = blockIdx.x; s < a.b; s += gridDim.x) {
+      if (clamp_len(__ldg(a.lens + s), a.m_max, nullptr, false) == 0) {
+        uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + int64_t(s) * a.h * kD);
+        for (int k = int(threadIdx.x) - 64; k < a.h * kD / 8; k += 256) o[k] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
 
   if (sc.t_begin < sc.t_end) {
     if (warp == 0) {
@@ -882,6 +890,8 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
 bool tc_supported(int d, int hq) { return d == kD && hq >= 1 && hq <= 64; }
 
 int tc_ctas_per_sm(int) { return 1; }
+
+int tc_tile_rows() { return kTile; }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) || int64_t(a.b) * a.h >= (int64_t(1) << 31))

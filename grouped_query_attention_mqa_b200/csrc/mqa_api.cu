@@ -121,6 +121,10 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.d = d_k;
   a.hq = hq;
   a.window = opts ? opts->window : 0;
+  // When no sequence spans more than one tile no segment is ever split, so
+  // every output row is final when the decode kernel ends: the merge is left out.
+  const int span_max = a.window > 0 && a.window < m_max ? a.window : m_max;
+  a.no_merge = span_max <= (use_tc ? tc_tile_rows() : simt_tile_rows());
   a.scale = scale;
   a.ws = carve_workspace(workspace, b, g, hq);
   a.flags = status_flags;
@@ -130,7 +134,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
 
   cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;
-  e = launch_merge(a, dtype, stream);
+  if (!a.no_merge) e = launch_merge(a, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;
   return MQA_OK;
 }

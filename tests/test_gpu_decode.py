@@ -264,3 +264,31 @@ def test_tensor_core_path_large_batches(b):
         ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, 1, wl.scale)
         assert_close(o, ref, "bf16", f"b={b} ctas={ctas}")
         assert (o[lens == 0] == 0).all()
+
+
+@pytest.mark.parametrize("path,h,m_max,window,dtype", [
+    ("tcgen05", 32, 128, 0, "bf16"),     # every sequence fits one 128-row tile
+    ("tcgen05", 8, 600, 100, "bf16"),    # long sequences, but a window of one tile
+    ("simt", 4, 64, 0, "bf16"),          # one 64-row SIMT tile
+    ("simt", 4, 300, 64, "f32"),
+])
+def test_single_tile_sequences_need_no_merge(path, h, m_max, window, dtype):
+    """When no sequence spans two tiles no segment can be split, the merge
+    kernel is left out and the decode writes every output row itself,
+    including the zero rows of empty sequences.  The output starts as NaN, so
+    a row left unwritten fails."""
+    b = 40
+    wl = small(dtype, b, h, 1, 128 if dtype == "bf16" else 64, m_max, 1, 1)
+    rng = np.random.default_rng(h + m_max)
+    lens = rng.integers(0, m_max + 1, size=b).astype(np.int32)
+    lens[::7] = 0
+    inp = host_inputs(wl, seed=m_max, nan_tail=True, lens=np.maximum(lens, 1))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    for ctas in (0, 1, 7, 300):
+        out = torch.full((b, h, wl.d_v), float("nan"), dtype=tdt, device="cuda")
+        binding.decode(dev(inp["q"], dtype), dev(inp["k"], dtype), dev(inp["v"], dtype), torch.from_numpy(lens).cuda(),
+                       wl.scale, out=out, path=path, num_ctas=ctas, window=window)
+        ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, 1, wl.scale, window=window)
+        o = host64(out)
+        assert_close(o, ref, dtype, f"{path} ctas={ctas}")
+        assert (o[lens == 0] == 0).all()
