@@ -4,4 +4,5 @@ from .mqa_oracle import (  # noqa: F401
     oracle_decode,
     oracle_decode_step,
     oracle_kv_append,
+    oracle_prefill,
 )

@@ -9,8 +9,10 @@ the pages, without blocking, splitting or reordering.
 Sources (web pages on Multi-Query Attention; cited by title and section):
 
 * [velog review] "[Paper review] Fast Transformer Decoding: One Write-Head is All
-  You Need", §2.1 (DotProductAttention), §2.4 (MultiheadSelfAttentionIncremental)
-  and §3 (MultiquerySelfAttentionIncremental).  These give the computation as
+  You Need", §2.1 (DotProductAttention), §2.3 (Multi-head Attention (Batched):
+  logits = einsum("bhnk,bhmk->bhnm"), softmax(logits + mask)), §2.4
+  (MultiheadSelfAttentionIncremental) and §3 (MultiquerySelfAttentionIncremental;
+  MQA drops the h axis of K/V).  These give the computation as
   einsums: logits = einsum("bhk,bmk->bhm", q, K); weights = softmax(logits);
   o = einsum("bhm,bmv->bhv", weights, V); the per-head form has K/V [b,h,m,k].
 * [kuangjux notes] "Fast Transformer Decoding: One Write-Head is All You Need"
@@ -33,6 +35,11 @@ notes of the repository):
 * Grouping: query head i reads K/V head j(i) = i // (h // g), i.e. contiguous
   groups; h must be a multiple of g.
 * lens[b] == 0: the output row is 0 and lse is -inf (the pages do not define it).
+* Prefill: the review's batched form takes a general additive mask [b,h,n,m];
+  the notes' §1 and §10 describe prefill as the whole prompt at once under a
+  causal mask.  Reading: with ``causal`` query position t of a sequence sees
+  the keys 0..t of the same sequence (mask 0, else -inf); without it, all keys
+  of the sequence.  Sequences are packed: rows cu_seqlens[s] .. cu_seqlens[s+1]-1.
 * Local window: the notes name a window of the current position plus the 31
   before it, with no formula.  With ``window`` = w > 0, position t of sequence
   b is attended iff lens[b] - w <= t < lens[b] (the newest w rows; w = 32 is the
@@ -52,6 +59,7 @@ __all__ = [
     "oracle_decode",
     "oracle_kv_append",
     "oracle_decode_step",
+    "oracle_prefill",
 ]
 
 
@@ -176,3 +184,49 @@ def oracle_decode_step(q, k_cache, v_cache, k_new, v_new, lens_before, g, scale,
     lens_after = np.asarray(lens_before).astype(np.int64) + 1
     o, lse = oracle_decode(q, k2, v2, lens_after, g, scale, window=window)
     return o, lse, k2, v2
+
+
+def oracle_prefill(q, k, v, cu_seqlens, g, scale, causal=True):
+    """Attention of every position of every sequence over the same sequence's
+    keys, in float64: the batched form of [velog review] §2.3 with the K/V head
+    axis removed as in §3 (h // g query heads per K/V head, [oscine blog]
+    "第三站: GQA"), under a causal mask for prefill ([kuangjux notes] §1, §10).
+
+    Shapes (packed sequences): q [T, h, d_k]; k [T, g, d_k]; v [T, g, d_v];
+    cu_seqlens int [b+1], sequence s holding rows cu_seqlens[s] .. cu_seqlens[s+1]-1.
+    Returns o [T, h, d_v] and lse [T, h] (natural log of the softmax denominator).
+
+    For each sequence and K/V group j, with Q_j [n, h//g, d_k] and K_j, V_j [n, d]:
+        S[t, i, u] = scale · Q_j[t, i] · K_j[u]          (§2.3 logits einsum)
+        S[t, i, u] = -inf for u > t when causal           (the mask)
+        W = softmax over u;  O[t, i] = Σ_u W[t, i, u] V_j[u]
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    cu = np.asarray(cu_seqlens).astype(np.int64)
+    T, h, d_k = q.shape
+    d_v = v.shape[2]
+    if k.shape[:2] != (T, g) or v.shape[:2] != (T, g) or h % g != 0:
+        raise ValueError("k/v must be [T, g, d] and h a multiple of g")
+    hq = h // g
+    o = np.zeros((T, h, d_v), dtype=np.float64)
+    lse = np.full((T, h), -np.inf, dtype=np.float64)
+    for si in range(len(cu) - 1):
+        a, e = int(cu[si]), int(cu[si + 1])
+        n = e - a
+        if n <= 0:
+            continue
+        allowed = np.tril(np.ones((n, n), dtype=bool)) if causal else np.ones((n, n), dtype=bool)   # [query, key]
+        for j in range(g):
+            Qj = q[a:e, j * hq:(j + 1) * hq, :].astype(np.float64)            # [n, hq, d_k]
+            Kj = k[a:e, j, :].astype(np.float64)                               # [n, d_k]
+            Vj = v[a:e, j, :].astype(np.float64)                               # [n, d_v]
+            S = scale * np.einsum("tik,uk->tiu", Qj, Kj)                       # [n, hq, n]
+            S = np.where(allowed[:, None, :], S, -np.inf)
+            mu = S.max(axis=2, keepdims=True)
+            E = np.exp(S - mu)
+            denom = E.sum(axis=2, keepdims=True)
+            o[a:e, j * hq:(j + 1) * hq, :] = np.einsum("tiu,uv->tiv", E / denom, Vj)
+            lse[a:e, j * hq:(j + 1) * hq] = (mu + np.log(denom))[:, :, 0]
+    return o, lse

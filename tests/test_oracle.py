@@ -412,3 +412,88 @@ def test_step_with_window_attends_the_appended_row():
     for bi in range(b):
         for i in range(h):
             np.testing.assert_array_equal(o[bi, i], vn[bi, i // (h // g)])
+
+
+# ------------------------------------------------------------ prefill (batched, causal)
+
+from oracle import oracle_prefill   # noqa: E402
+
+
+def _packed(rng, lens, h, g, d):
+    T = int(sum(lens))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return _rand(rng, T, h, d), _rand(rng, T, g, d), _rand(rng, T, g, d), cu
+
+
+@pytest.mark.parametrize("h,g", [(4, 1), (4, 2), (4, 4)])
+def test_prefill_is_brute_force_over_the_causal_prefix(h, g):
+    """Query t of a sequence is DotProductAttention ([velog review] §2.1) over
+    keys 0..t of the same sequence: the review's batched form with a causal
+    mask."""
+    rng = np.random.default_rng(60 + h + g)
+    lens = [5, 1, 3]
+    q, k, v, cu = _packed(rng, lens, h, g, 3)
+    o, _ = oracle_prefill(q, k, v, cu, g=g, scale=0.8)
+    for si, n in enumerate(lens):
+        a = int(cu[si])
+        for t in range(n):
+            for i in range(h):
+                j = i // (h // g)
+                y, _ = dot_product_attention(q[a + t, i], k[a:a + t + 1, j], v[a:a + t + 1, j], scale=0.8)
+                np.testing.assert_allclose(o[a + t, i], y, rtol=0, atol=1e-13)
+
+
+def test_prefill_first_position_returns_its_own_v():
+    """The causal mask leaves one key for position 0: o = v[0] exactly."""
+    rng = np.random.default_rng(61)
+    q, k, v, cu = _packed(rng, [4, 6], 4, 2, 5)
+    o, lse = oracle_prefill(q, k, v, cu, g=2, scale=1.3)
+    for a in (0, 4):
+        for i in range(4):
+            np.testing.assert_array_equal(o[a, i], v[a, i // 2])
+            np.testing.assert_allclose(lse[a, i], 1.3 * float(q[a, i] @ k[a, i // 2]), rtol=0, atol=1e-13)
+
+
+def test_prefill_without_mask_sees_the_whole_sequence():
+    rng = np.random.default_rng(62)
+    lens = [4, 3]
+    q, k, v, cu = _packed(rng, lens, 2, 1, 3)
+    o, _ = oracle_prefill(q, k, v, cu, g=1, scale=1.0, causal=False)
+    for si, n in enumerate(lens):
+        a = int(cu[si])
+        for t in range(n):
+            for i in range(2):
+                y, _ = dot_product_attention(q[a + t, i], k[a:a + n, 0], v[a:a + n, 0], scale=1.0)
+                np.testing.assert_allclose(o[a + t, i], y, rtol=0, atol=1e-13)
+
+
+def test_prefill_prefix_is_unchanged_by_later_tokens():
+    """Causality: outputs of positions 0..n-1 do not depend on tokens appended
+    after them."""
+    rng = np.random.default_rng(63)
+    q, k, v, cu = _packed(rng, [9], 4, 1, 4)
+    o_full, _ = oracle_prefill(q, k, v, cu, g=1, scale=1.0)
+    o_cut, _ = oracle_prefill(q[:5], k[:5], v[:5], [0, 5], g=1, scale=1.0)
+    np.testing.assert_allclose(o_full[:5], o_cut, rtol=0, atol=1e-15)
+
+
+def test_prefill_last_position_is_the_decode_step():
+    """The last position of a prefill attends to the whole sequence, exactly as
+    one decode step over a cache holding that sequence."""
+    rng = np.random.default_rng(64)
+    lens = [7, 2]
+    q, k, v, cu = _packed(rng, lens, 6, 3, 4)
+    o, lse = oracle_prefill(q, k, v, cu, g=3, scale=0.5)
+    for si, n in enumerate(lens):
+        a = int(cu[si])
+        od, lsed = oracle_decode(q[a + n - 1][None], k[a:a + n][None], v[a:a + n][None], [n], g=3, scale=0.5)
+        np.testing.assert_allclose(o[a + n - 1], od[0], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[a + n - 1], lsed[0], rtol=0, atol=1e-13)
+
+
+def test_prefill_mqa_equals_mha_with_replicated_kv():
+    rng = np.random.default_rng(65)
+    q, k, v, cu = _packed(rng, [6, 3], 4, 1, 3)
+    o1, _ = oracle_prefill(q, k, v, cu, g=1, scale=1.0)
+    o4, _ = oracle_prefill(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), cu, g=4, scale=1.0)
+    np.testing.assert_allclose(o1, o4, rtol=0, atol=1e-15)
