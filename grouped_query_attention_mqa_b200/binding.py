@@ -44,6 +44,8 @@ SIGNATURES = {
                                    ctypes.POINTER(DecodeOptions), _c_ptr]),
     "mqa_decode_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
                                     _c_int, _c_float, _c_int, _c_ptr, _c_ptr]),
+    "mqa_prefill": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                             _c_int, _c_float, _c_int, _c_int, _c_ptr, _c_ptr]),
     "mqa_status_string": (ctypes.c_char_p, [_c_int]),
 }
 
@@ -182,6 +184,34 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
                              _ptr(status_flags), ctypes.byref(opts), _stream_handle(stream))
     if st != MQA_OK:
         raise MqaError(st, "mqa_decode")
+    return out
+
+
+def prefill(q, k, v, cu_seqlens, max_seqlen, scale, causal=True, out=None, status_flags=None, stream=None):
+    """Batched (prefill) attention over packed sequences (mqa_prefill): q [T,h,d],
+    k/v [T,g,d], cu_seqlens int32 [b+1] on the device, max_seqlen the longest
+    sequence.  Returns o [T,h,d]."""
+    import torch
+    _check_cuda(q, k, v, cu_seqlens, out, status_flags)
+    T, h, d_k = q.shape
+    if tuple(k.shape[:1]) != (T,) or k.shape[0] != v.shape[0] or k.shape[1] != v.shape[1]:
+        raise ValueError("prefill: k/v must be [T,g,d] with q's T")
+    g = k.shape[1]
+    d_v = v.shape[2]
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be int32 [b+1]")
+    dt = _dtype_code(q)
+    if any(_dtype_code(t) != dt for t in (k, v)):
+        raise TypeError("prefill: q, k and v must share one dtype")
+    if out is None:
+        out = torch.empty((T, h, d_v), dtype=q.dtype, device=q.device)
+    elif tuple(out.shape) != (T, h, d_v) or out.dtype != q.dtype:
+        raise ValueError("prefill: out must be [T,h,d_v] in q's dtype")
+    st = lib().mqa_prefill(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
+                           int(max_seqlen), h, g, d_k, d_v, float(scale), 1 if causal else 0, dt, _ptr(status_flags),
+                           _stream_handle(stream))
+    if st != MQA_OK:
+        raise MqaError(st, "mqa_prefill")
     return out
 
 

@@ -485,6 +485,10 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStrea
 int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq);
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+bool prefill_tc_supported(int d, int hq);
+cudaError_t launch_prefill_tc(void* o, const void* q, const void* k, const void* v, const int32_t* cu, int b,
+                              int64_t total, int h, int g, int max_seqlen, float scale, int causal, int32_t* flags,
+                              cudaStream_t stream);
 int tc_ctas_per_sm(int hq);
 int tc_tile_rows();
 int simt_tile_rows();

@@ -151,6 +151,23 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
                      workspace, workspace_bytes_given, status_flags, opts, stream);
 }
 
+mqa_status_t mqa_prefill(void* o, const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int b,
+                         int total, int max_seqlen, int h, int g, int d_k, int d_v, float scale, int causal,
+                         mqa_dtype_t dtype, int32_t* status_flags, cudaStream_t stream) {
+  if (b < 0 || total < 0 || max_seqlen < 0 || h < 1 || g < 1 || h % g != 0 || d_k < 1 || d_v < 1 ||
+      !valid_dtype(dtype) || !std::isfinite(scale) || (causal != 0 && causal != 1))
+    return MQA_ERR_INVALID_ARG;
+  if (b == 0 || total == 0 || max_seqlen == 0) return MQA_OK;
+  if (!o || !q || !k || !v || !cu_seqlens) return MQA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(cu_seqlens))
+    return MQA_ERR_INVALID_ARG;
+  if (dtype != MQA_BF16 || d_k != d_v || !prefill_tc_supported(d_k, h / g)) return MQA_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_prefill_tc(o, q, k, v, cu_seqlens, b, total, h, g, max_seqlen, scale, causal,
+                                          status_flags, stream);
+  if (e == cudaErrorInvalidValue) return MQA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? MQA_OK : MQA_ERR_CUDA;
+}
+
 mqa_status_t mqa_decode(void* o, const void* q, const void* k_cache, const void* v_cache, const int32_t* lens, int b,
                         int h, int g, int m_max, int d_k, int d_v, float scale, mqa_dtype_t dtype, void* workspace,
                         size_t workspace_bytes_given, int32_t* status_flags, cudaStream_t stream) {

@@ -231,6 +231,39 @@ MQA_API mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k_ca
                                         float scale, mqa_dtype_t dtype, int32_t* status_flags,
                                         cudaStream_t stream);
 
+/*
+ * mqa_prefill — batched (prefill) attention: every position of every
+ * sequence attends to the keys of its own sequence.
+ *
+ * Source: the paper review of "Fast Transformer Decoding", §2.3 Multi-head
+ * Attention (Batched): logits = einsum("bhnk,bhmk->bhnm", Q, K),
+ * weights = softmax(logits + mask), O = einsum("bhnm,bhmv->bhnv", weights, V),
+ * with the K/V head axis removed as in §3 (h/g query heads per K/V head); the
+ * study notes on the same paper, §1 and §10, describe prefill as the whole
+ * prompt at once under a causal mask.  Here the mask is causal (causal = 1:
+ * position t sees keys 0..t of its sequence) or absent (causal = 0: all keys
+ * of the sequence), and sequences are packed without padding:
+ *
+ *   o           device [total, h, d_v]   written for every row of a sequence
+ *   q           device [total, h, d_k]
+ *   k, v        device [total, g, d_k], [total, g, d_v]
+ *   cu_seqlens  device int32 [b+1]: sequence s holds rows
+ *               cu_seqlens[s] .. cu_seqlens[s+1]-1 (non-decreasing, from 0)
+ *   max_seqlen  host: the longest sequence; the launch covers that many
+ *               positions per sequence
+ *   scale       multiplies the logits (e.g. 1/sqrt(d_k))
+ *
+ * Row-major, contiguous, 16-byte aligned, caller-owned.  Only bf16 with
+ * d_k = d_v = 128 and h/g dividing 128 is built (tensor-core path); other
+ * shapes return MQA_ERR_UNSUPPORTED before any launch.  A length read on the
+ * device that exceeds max_seqlen or runs past `total` rows is cut there and
+ * MQA_FLAG_LEN_CLAMPED is set; rows outside the arrays are never touched.
+ * Bounded waits report MQA_FLAG_PIPE_TIMEOUT.  Asynchronous on `stream`.
+ */
+MQA_API mqa_status_t mqa_prefill(void* o, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                 int b, int total, int max_seqlen, int h, int g, int d_k, int d_v, float scale,
+                                 int causal, mqa_dtype_t dtype, int32_t* status_flags, cudaStream_t stream);
+
 /* Static, NUL-terminated name of a status code. */
 MQA_API const char* mqa_status_string(mqa_status_t status);
 

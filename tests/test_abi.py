@@ -26,7 +26,7 @@ def header_symbols():
 def test_header_declares_the_boundary():
     assert header_symbols() == sorted(["mqa_kv_append", "mqa_decode_workspace_size", "mqa_decode",
                                        "mqa_decode_ex", "mqa_decode_append", "mqa_decode_noalloc",
-                                       "mqa_status_string"])
+                                       "mqa_prefill", "mqa_status_string"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -113,3 +113,28 @@ def test_append_rejects_bad_arguments_without_launching(lib):
 def test_binding_fails_loudly_without_the_library(tmp_path):
     with pytest.raises(RuntimeError, match="not built"):
         binding.load_library(str(tmp_path / "libmqa.so"))
+
+
+def _prefill(lib, **kw):
+    a = dict(o=FAKE, q=FAKE, k=FAKE, v=FAKE, cu=FAKE, b=2, total=64, max_seqlen=40, h=8, g=1, d_k=128, d_v=128,
+             scale=1.0, causal=1, dtype=binding.MQA_BF16, flags=None, stream=None)
+    a.update(kw)
+    return lib.mqa_prefill(a["o"], a["q"], a["k"], a["v"], a["cu"], a["b"], a["total"], a["max_seqlen"], a["h"],
+                           a["g"], a["d_k"], a["d_v"], a["scale"], a["causal"], a["dtype"], a["flags"], a["stream"])
+
+
+def test_prefill_rejects_bad_arguments_without_launching(lib):
+    INV, UNS = binding.MQA_ERR_INVALID_ARG, binding.MQA_ERR_UNSUPPORTED
+    assert _prefill(lib, g=3) == INV                     # h % g != 0
+    assert _prefill(lib, q=None) == INV
+    assert _prefill(lib, cu=None) == INV
+    assert _prefill(lib, o=ctypes.c_void_p(0x10008)) == INV
+    assert _prefill(lib, total=-1) == INV
+    assert _prefill(lib, max_seqlen=-1) == INV
+    assert _prefill(lib, causal=2) == INV
+    assert _prefill(lib, scale=float("nan")) == INV
+    assert _prefill(lib, dtype=binding.MQA_F32) == UNS   # only bf16 is built
+    assert _prefill(lib, d_k=64, d_v=64) == UNS          # only d = 128
+    assert _prefill(lib, h=12, g=1) == UNS               # h/g must divide 128
+    assert _prefill(lib, b=0) == binding.MQA_OK          # nothing to do
+    assert _prefill(lib, total=0) == binding.MQA_OK
