@@ -29,9 +29,10 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from grouped_query_attention_mqa_b200.workloads import (WORKLOADS, append_algorithmic_bytes,  # noqa: E402
-                                                         decode_algorithmic_bytes, draw_lens, f32_to_bf16_bits,
-                                                         bf16_bits_to_f32)
+from grouped_query_attention_mqa_b200.workloads import (PREFILL_WORKLOADS, WORKLOADS,  # noqa: E402
+                                                         append_algorithmic_bytes, decode_algorithmic_bytes,
+                                                         draw_lens, f32_to_bf16_bits, bf16_bits_to_f32,
+                                                         prefill_flops)
 
 METRIC = "decode-attention achieved HBM GB/s vs peak; query-tokens/s at MQA b=64 m=8K"
 UNIT = "query-tokens/s"
@@ -46,7 +47,7 @@ def parse():
     p.add_argument("--steps", type=int, default=20000)
     p.add_argument("--warmup", type=int, default=200)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
     p.add_argument("--num-ctas", type=int, default=0)
     p.add_argument("--window", type=int, default=0, help="local attention: attend to the newest W rows (0 = all)")
@@ -466,9 +467,159 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ prefill
+
+PREFILL_METRIC = "batched (prefill) attention TFLOP/s"
+
+
+def time_oracle_prefill(wl, seconds, n=512):
+    """The prefill oracle on one sequence of n tokens of the workload's shape,
+    repeated until about `seconds` of CPU time; returns (FLOP/s, runs, s)."""
+    from oracle import oracle_prefill   # test infrastructure: only the CPU legs of the bench run it
+    rng = np.random.default_rng(SEED)
+    q = bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((n, wl.h, wl.d), dtype=np.float32)))
+    k = bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((n, wl.g, wl.d), dtype=np.float32)))
+    v = bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((n, wl.g, wl.d), dtype=np.float32)))
+    pairs = n * (n + 1) // 2 if wl.causal else n * n
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle_prefill(q, k, v, [0, n], wl.g, wl.scale, causal=wl.causal)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done * 4 * wl.h * wl.d * pairs / el, done, el
+
+
+def run_prefill(args):
+    """mqa_prefill on packed equal-length sequences: TFLOP/s of the attention
+    (4 h d FLOPs per attended pair) against the measured bf16 tensor peak."""
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = PREFILL_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            time_oracle_prefill(wl, 0.0, n=128)
+        rates, runs, total = [], 0, 0.0
+        for _ in range(args.steps):
+            r, n_runs, el = time_oracle_prefill(wl, per)
+            rates.append(r)
+            runs += n_runs
+            total += el
+        value = float(np.median(rates)) / 1e12
+        print(json.dumps({"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s",
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "config": {"workload": wl.name}, "data": "synthetic",
+                          "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                                           "kind": "oracle",
+                                           "sample": f"{runs} runs of one 512-token sequence of {wl.name}'s shape, "
+                                                     f"NumPy float64, {total:.1f} s"},
+                          "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from grouped_query_attention_mqa_b200 import binding
+    from grouped_query_attention_mqa_b200.build import LIB, build
+    from grouped_query_attention_mqa_b200.workloads import prefill_device_inputs
+    if not os.path.exists(LIB):
+        build()
+    binding.load_library()
+    inp = prefill_device_inputs(wl, seed=rank_seed(rank), device="cuda")
+    out = torch.empty_like(inp["q"])
+    flops = prefill_flops(wl)
+
+    def step():
+        binding.prefill(inp["q"], inp["k"], inp["v"], inp["cu"], wl.n, wl.scale, causal=wl.causal, out=out)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    time.sleep(0.2)
+    start.record()
+    for _ in range(K):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    elapsed_ms = reduce_over_ranks([start.elapsed_time(end)], "cuda")[0]
+    ms = elapsed_ms / K
+    tflops = flops / (ms / 1e3) / 1e12
+    value = tflops * world
+
+    # end to end: q, k, v copied in from pinned host memory and o copied out, every step
+    host = {name: inp[name].cpu().pin_memory() for name in ("q", "k", "v")}
+    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {name: torch.empty_like(inp[name]) for name in ("q", "k", "v")}
+    E = max(3, min(args.e2e_steps, 50))
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(E):
+        for name in ("q", "k", "v"):
+            dev_in[name].copy_(host[name], non_blocking=True)
+        binding.prefill(dev_in["q"], dev_in["k"], dev_in["v"], inp["cu"], wl.n, wl.scale, causal=wl.causal, out=out)
+        o_h.copy_(out, non_blocking=True)
+    e2.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_over_ranks([s2.elapsed_time(e2)], "cuda")[0] / E
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size()
+    pk = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            pk = json.load(fh).get("bf16_tflops")
+    except OSError:
+        pass
+    peak, peak_kind = (float(pk), "measured") if pk else (1590.0, "fallback")
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            r, runs, el = time_oracle_prefill(wl, args.cpu_seconds)
+            cpu = {"value": r / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{runs} runs of one 512-token sequence of {wl.name}'s shape, NumPy float64, {el:.1f} s"}
+        print(json.dumps({
+            "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "b": wl.b, "n": wl.n, "h": wl.h, "g": wl.g, "d": wl.d,
+                       "causal": wl.causal, "tokens_per_s": wl.total * world / (ms / 1e3),
+                       "l2": "q and o (2 x %d MiB) exceed the L2; K/V tiles are meant to be reused from it"
+                             % (inp["q"].numel() * 2 // 2**20),
+                       "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "prefill_tc_kernel, average over the timed steps",
+                         "algorithmic_flops_per_launch": flops, "launch_ms": ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": E},
+            "gpu_launches": K,
+            "clocks": clk,
+        }), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.workload in PREFILL_WORKLOADS:
+        run_prefill(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -222,3 +222,52 @@ def decode_flops(wl: Workload, lens) -> int:
     """2·d_k FLOPs per (head, row) for q·k plus 2·d_v for the weighted V."""
     lens = np.asarray(lens, dtype=np.int64)
     return int(lens.sum()) * wl.h * 2 * (wl.d_k + wl.d_v)
+
+
+@dataclass(frozen=True)
+class PrefillWorkload:
+    """One batched (prefill) attention problem: b sequences of n tokens each,
+    packed, h query heads sharing g K/V heads of size d, causal or not."""
+    name: str
+    b: int
+    n: int
+    h: int
+    g: int
+    d: int
+    causal: bool
+    scale: float
+    description: str = ""
+
+    @property
+    def total(self) -> int:
+        return self.b * self.n
+
+
+PREFILL_WORKLOADS = {
+    "prefill_mqa_b8_n4096": PrefillWorkload(
+        "prefill_mqa_b8_n4096", b=8, n=4096, h=32, g=1, d=128, causal=True, scale=_S128,
+        description="MQA prompt prefill: 8 sequences x 4096 tokens, h=32 g=1 d=128, causal"),
+    "prefill_gqa8_b4_n8192": PrefillWorkload(
+        "prefill_gqa8_b4_n8192", b=4, n=8192, h=64, g=8, d=128, causal=True, scale=_S128,
+        description="GQA-8 prompt prefill: 4 sequences x 8192 tokens, h=64 g=8 d=128, causal"),
+}
+
+
+def prefill_flops(wl: PrefillWorkload) -> int:
+    """2 h d FLOPs for q.k and 2 h d for p.v per attended (query, key) pair."""
+    pairs = wl.n * (wl.n + 1) // 2 if wl.causal else wl.n * wl.n
+    return 4 * wl.h * wl.d * pairs * wl.b
+
+
+def prefill_device_inputs(wl: PrefillWorkload, seed: int, device):
+    """q [T,h,d], k/v [T,g,d] bf16 N(0,1) from torch's seeded generator, and
+    cu_seqlens int32 [b+1] for equal-length packed sequences."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    T = wl.total
+    out = {}
+    for name, heads in (("q", wl.h), ("k", wl.g), ("v", wl.g)):
+        out[name] = torch.randn((T, heads, wl.d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    out["cu"] = torch.arange(0, T + 1, wl.n, dtype=torch.int32, device=device)
+    return out
