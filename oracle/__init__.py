@@ -5,4 +5,5 @@ from .mqa_oracle import (  # noqa: F401
     oracle_decode_step,
     oracle_kv_append,
     oracle_prefill,
+    oracle_decode_beam,
 )

@@ -40,6 +40,10 @@ notes of the repository):
   causal mask.  Reading: with ``causal`` query position t of a sequence sees
   the keys 0..t of the same sequence (mask 0, else -inf); without it, all keys
   of the sequence.  Sequences are packed: rows cu_seqlens[s] .. cu_seqlens[s+1]-1.
+* Beam search: the notes' §6.2 and §6.4 time a beam-4 decoder but give no
+  formula.  Reading: each of W beams of a sequence attends over the
+  sequence's shared prefix rows followed by its own suffix rows (the tokens
+  that beam generated), i.e. plain decode attention over that concatenation.
 * Local window: the notes name a window of the current position plus the 31
   before it, with no formula.  With ``window`` = w > 0, position t of sequence
   b is attended iff lens[b] - w <= t < lens[b] (the newest w rows; w = 32 is the
@@ -60,6 +64,7 @@ __all__ = [
     "oracle_kv_append",
     "oracle_decode_step",
     "oracle_prefill",
+    "oracle_decode_beam",
 ]
 
 
@@ -229,4 +234,37 @@ def oracle_prefill(q, k, v, cu_seqlens, g, scale, causal=True):
             denom = E.sum(axis=2, keepdims=True)
             o[a:e, j * hq:(j + 1) * hq, :] = np.einsum("tiu,uv->tiv", E / denom, Vj)
             lse[a:e, j * hq:(j + 1) * hq] = (mu + np.log(denom))[:, :, 0]
+    return o, lse
+
+
+def oracle_decode_beam(q, prefix_k, prefix_v, prefix_lens, suffix_k, suffix_v, suffix_lens, g, scale):
+    """One decode step of W beams per sequence that share a prefix, in float64
+    ([kuangjux notes] §6.2/§6.4 beam-4 decoding; reading in the header).
+
+    Shapes: q [b, W, h, d_k]; prefix_k/v [b, m_p, g, d]; prefix_lens [b];
+    suffix_k/v [b*W, m_s, g, d] (beam w of sequence s at row s*W + w);
+    suffix_lens [b*W].  Beam (s, w) attends over prefix rows 0..prefix_lens[s]-1
+    of sequence s followed by suffix rows 0..suffix_lens[s*W+w]-1 of its own
+    cache: oracle_decode on that concatenated cache.  Returns o [b, W, h, d_v]
+    and lse [b, W, h].
+    """
+    q = np.asarray(q)
+    b, W, h, d_k = q.shape
+    pk, pv = np.asarray(prefix_k), np.asarray(prefix_v)
+    sk, sv = np.asarray(suffix_k), np.asarray(suffix_v)
+    lp = np.asarray(prefix_lens).astype(np.int64)
+    ls = np.asarray(suffix_lens).astype(np.int64)
+    d_v = pv.shape[3]
+    o = np.zeros((b, W, h, d_v), dtype=np.float64)
+    lse = np.full((b, W, h), -np.inf, dtype=np.float64)
+    for si in range(b):
+        for w in range(W):
+            r = si * W + w
+            K = np.concatenate([pk[si, :lp[si]], sk[r, :ls[r]]], axis=0)[None]     # [1, L, g, d]
+            V = np.concatenate([pv[si, :lp[si]], sv[r, :ls[r]]], axis=0)[None]
+            L = K.shape[1]
+            if L == 0:
+                continue
+            ob, lb = oracle_decode(q[si, w][None], K, V, [L], g, scale)
+            o[si, w], lse[si, w] = ob[0], lb[0]
     return o, lse

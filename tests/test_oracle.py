@@ -497,3 +497,58 @@ def test_prefill_mqa_equals_mha_with_replicated_kv():
     o1, _ = oracle_prefill(q, k, v, cu, g=1, scale=1.0)
     o4, _ = oracle_prefill(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), cu, g=4, scale=1.0)
     np.testing.assert_allclose(o1, o4, rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------ beams sharing a prefix
+
+from oracle import oracle_decode_beam   # noqa: E402
+
+
+def _beam_problem(rng, b, W, h, g, d, mp, ms):
+    return (_rand(rng, b, W, h, d), _rand(rng, b, mp, g, d), _rand(rng, b, mp, g, d),
+            _rand(rng, b * W, ms, g, d), _rand(rng, b * W, ms, g, d))
+
+
+def test_beam_is_brute_force_over_prefix_then_suffix():
+    """Beam (s, w), head i: DotProductAttention ([velog review] §2.1) over the
+    shared prefix rows of sequence s followed by the beam's own suffix rows."""
+    rng = np.random.default_rng(70)
+    b, W, h, g, d = 2, 3, 4, 2, 3
+    q, pk, pv, sk, sv = _beam_problem(rng, b, W, h, g, d, 6, 4)
+    lp, ls = [5, 2], [0, 1, 4, 3, 2, 0]
+    o, _ = oracle_decode_beam(q, pk, pv, lp, sk, sv, ls, g=g, scale=0.6)
+    for si in range(b):
+        for w in range(W):
+            r = si * W + w
+            for i in range(h):
+                j = i // (h // g)
+                K = np.concatenate([pk[si, :lp[si], j], sk[r, :ls[r], j]])
+                V = np.concatenate([pv[si, :lp[si], j], sv[r, :ls[r], j]])
+                y, _ = dot_product_attention(q[si, w, i], K, V, scale=0.6)
+                np.testing.assert_allclose(o[si, w, i], y, rtol=0, atol=1e-13)
+
+
+def test_beams_with_the_same_suffix_agree():
+    """Beams are independent rows: equal queries and equal suffixes give equal outputs."""
+    rng = np.random.default_rng(71)
+    q, pk, pv, sk, sv = _beam_problem(rng, 1, 4, 2, 1, 3, 5, 3)
+    q[0, :] = q[0, 0]
+    sk[:] = sk[0]
+    sv[:] = sv[0]
+    o, _ = oracle_decode_beam(q, pk, pv, [5], sk, sv, [2, 2, 2, 2], g=1, scale=1.0)
+    for w in range(1, 4):
+        np.testing.assert_array_equal(o[0, w], o[0, 0])
+
+
+def test_beam_with_empty_suffix_or_prefix_is_plain_decode():
+    """No suffix rows: decode over the prefix; no prefix rows: decode over the suffix."""
+    rng = np.random.default_rng(72)
+    q, pk, pv, sk, sv = _beam_problem(rng, 2, 2, 4, 1, 3, 7, 5)
+    o, lse = oracle_decode_beam(q, pk, pv, [7, 3], sk, sv, [0, 0, 0, 0], g=1, scale=1.0)
+    od, lsed = oracle_decode(q.reshape(4, 4, 3), np.repeat(pk, 2, axis=0), np.repeat(pv, 2, axis=0),
+                             [7, 7, 3, 3], g=1, scale=1.0)
+    np.testing.assert_allclose(o.reshape(4, 4, 3), od, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse.reshape(4, 4), lsed, rtol=0, atol=1e-14)
+    o, _ = oracle_decode_beam(q, pk, pv, [0, 0], sk, sv, [5, 1, 2, 3], g=1, scale=1.0)
+    od, _ = oracle_decode(q.reshape(4, 4, 3), sk, sv, [5, 1, 2, 3], g=1, scale=1.0)
+    np.testing.assert_allclose(o.reshape(4, 4, 3), od, rtol=0, atol=1e-15)
