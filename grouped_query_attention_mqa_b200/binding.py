@@ -44,6 +44,10 @@ SIGNATURES = {
                                    ctypes.POINTER(DecodeOptions), _c_ptr]),
     "mqa_decode_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int,
                                     _c_int, _c_float, _c_int, _c_ptr, _c_ptr]),
+    "mqa_decode_beam_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "mqa_decode_beam": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_ptr, _c_size,
+                                 _c_ptr, _c_ptr]),
     "mqa_prefill": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                              _c_int, _c_float, _c_int, _c_int, _c_ptr, _c_ptr]),
     "mqa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -184,6 +188,37 @@ def decode(q, k_cache, v_cache, lens, scale, out=None, workspace=None, status_fl
                              _ptr(status_flags), ctypes.byref(opts), _stream_handle(stream))
     if st != MQA_OK:
         raise MqaError(st, "mqa_decode")
+    return out
+
+
+def decode_beam(q, prefix_k, prefix_v, prefix_lens, suffix_k, suffix_v, suffix_lens, scale, out=None,
+                workspace=None, status_flags=None, stream=None):
+    """One decode step of W beams sharing each sequence's prefix
+    (mqa_decode_beam): q [b,W,h,d]; prefix caches [b,m_p,g,d] with lens [b];
+    suffix caches [b*W,m_s,g,d] with lens [b*W].  Returns o [b,W,h,d]."""
+    import torch
+    _check_cuda(q, prefix_k, prefix_v, prefix_lens, suffix_k, suffix_v, suffix_lens, out, workspace, status_flags)
+    b, W, h, d_k = q.shape
+    _, m_p, g, _ = prefix_k.shape
+    m_s = suffix_k.shape[1]
+    d_v = prefix_v.shape[3]
+    if tuple(prefix_k.shape) != (b, m_p, g, d_k) or tuple(suffix_k.shape) != (b * W, m_s, g, d_k):
+        raise ValueError("decode_beam: inconsistent cache shapes")
+    if prefix_lens.dtype != torch.int32 or suffix_lens.dtype != torch.int32 or prefix_lens.numel() != b \
+            or suffix_lens.numel() != b * W:
+        raise ValueError("decode_beam: lens must be int32 [b] and [b*W]")
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((b, W, h, d_v), dtype=q.dtype, device=q.device)
+    need = lib().mqa_decode_beam_workspace_size(b, W, h, g, d_v)
+    if workspace is None:
+        workspace = torch.empty(max(256, need), dtype=torch.uint8, device=q.device)
+    st = lib().mqa_decode_beam(_ptr(out), _ptr(q), _ptr(prefix_k), _ptr(prefix_v), _ptr(prefix_lens), _ptr(suffix_k),
+                               _ptr(suffix_v), _ptr(suffix_lens), b, W, h, g, m_p, m_s, d_k, d_v, float(scale), dt,
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status_flags),
+                               _stream_handle(stream))
+    if st != MQA_OK:
+        raise MqaError(st, "mqa_decode_beam")
     return out
 
 

@@ -472,6 +472,10 @@ struct DecodeArgs {
   int window;          // local attention: the newest `window` rows (0 = all rows)
   int no_merge;        // no segment spans two tiles: the decode writes every output row
                        // itself (zero rows for empty sequences) and no merge follows
+  int q_beams;         // 0: q is [b, h, d]; W > 0: q is [b, W, h, d] and a segment's query rows
+                       // are the W beams' q_group_heads heads of its group (hq = W * q_group_heads)
+  int q_group_heads;   // query heads per K/V head in q
+  int emit_partials;   // every segment leaves a partial and seg_info; o is not written
   float scale;
   Workspace ws;
   int32_t* flags;
@@ -485,6 +489,14 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStrea
 int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq);
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+struct BeamCombineArgs {
+  void* o;                    // [b, W, h, d] bf16
+  const int32_t* plens;       // [b] prefix lengths
+  const int32_t* slens;       // [b*W] suffix lengths
+  int b, W, h, g, hq, d, m_p, m_s;
+  Workspace pre, suf;         // partials of the prefix and the suffix pass
+};
+cudaError_t launch_beam_combine(const BeamCombineArgs& c, cudaStream_t stream);
 bool prefill_tc_supported(int d, int hq);
 cudaError_t launch_prefill_tc(void* o, const void* q, const void* k, const void* v, const int32_t* cu, int b,
                               int64_t total, int h, int g, int max_seqlen, float scale, int causal, int32_t* flags,

@@ -251,6 +251,24 @@ struct TileWalk {
   }
 };
 
+// Q of segment (seq, head) into a Q buffer (two 64-column halves of NP rows):
+// rows seq*h + head*hq.. of the 2-D map (d, b*h), or with beams the W beams'
+// q_group_heads heads of the group through the 3-D map (d, h, b*W).
+__device__ __forceinline__ void load_q(const DecodeArgs& a, const CUtensorMap* tm_q, uint32_t qdst, uint32_t bar,
+                                       int seq, int head, int np) {
+  if (a.q_beams > 0) {
+    const uint64_t pol = l2_evict_first_policy();
+    mbar_expect_tx(bar, 2u * uint32_t(a.hq) * 128u);
+    tma_load_3d(qdst, tm_q, bar, 0, head * a.q_group_heads, seq * a.q_beams, pol);
+    tma_load_3d(qdst + np * 128, tm_q, bar, 64, head * a.q_group_heads, seq * a.q_beams, pol);
+  } else {
+    mbar_expect_tx(bar, 2u * uint32_t(np) * 128u);
+    const int qrow = seq * a.h + head * a.hq;
+    tma_load_2d(qdst, tm_q, bar, 0, qrow);
+    tma_load_2d(qdst + np * 128, tm_q, bar, 64, qrow);
+  }
+}
+
 // Fused append: write the step's new row of (sequence, K/V head) into the
 // cache at row len-1, then order that store before the tensor-memory-access
 // read of the same row.
@@ -278,11 +296,7 @@ __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap*
   static_assert(SK >= 2 && SV >= 2, "two stages of each ring");
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  const int qrow = seq * a.h + head * a.hq;
-  const uint32_t qdst = r.sbase + C::kQ;
-  mbar_expect_tx(bar(C::kQFull), 2 * NP * 128);
-  tma_load_2d(qdst, tm_q, bar(C::kQFull), 0, qrow);
-  tma_load_2d(qdst + NP * 128, tm_q, bar(C::kQFull), 64, qrow);
+  load_q(a, tm_q, r.sbase + C::kQ, bar(C::kQFull), seq, head, NP);
   const int npre = own < 2 ? own : 2;
   for (int i = 0; i < npre; ++i) {
     const int k = k0 + i;
@@ -334,11 +348,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     if (kIsK && w.first) {
       const int qb = w.sidx & 1;
       if (w.sidx >= 2 && !wait_bar(r, bar(C::kQEmpty + qb), ((w.sidx >> 1) - 1) & 1)) break;
-      mbar_expect_tx(bar(C::kQFull + qb), 2 * NP * 128);
-      const int qrow = w.tc.seq * a.h + w.tc.head * a.hq;
-      const uint32_t qdst = r.sbase + C::kQ + qb * C::kQBytes;
-      tma_load_2d(qdst, tm_q, bar(C::kQFull + qb), 0, qrow);
-      tma_load_2d(qdst + NP * 128, tm_q, bar(C::kQFull + qb), 64, qrow);
+      load_q(a, tm_q, r.sbase + C::kQ + qb * C::kQBytes, bar(C::kQFull + qb), w.tc.seq, w.tc.head, NP);
       q_issued = w.sidx;
     }
     const int st = int(i % S);
@@ -520,7 +530,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     const int64_t slot = partial_slot(blockIdx.x, e.seg);
     float v[CPT];
     tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
-    if (e.whole) {
+    if (e.whole && !a.emit_partials) {
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) +
                            (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * kD + row;
 #pragma unroll
@@ -533,7 +543,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
         if (col0 + k < hq) dst[k * kD] = v[k] * linv[pb * NP + col0 + k];
     }
     if (warp == 2) {
-      if (!e.whole)
+      if (!e.whole || a.emit_partials)   // every partial carries its log-sum-exp
         for (int col = lane; col < hq; col += 32) a.ws.part_lse[slot * hq + col] = lse2[pb * NP + col];
       if (e.owns_first && lane == 0)
         a.ws.seg_info[e.seg] = make_int2(blockIdx.x, cta_of_unit(e.seg_last_unit, ws.wtotal, sc.active));
@@ -845,6 +855,17 @@ bool encode_cache(CUtensorMap* m, const void* base, int b, int m_max, int g) {
 }
 
 // q [b*h, 128] bf16; a box is 64 columns of NP consecutive heads.
+// Beam queries [b*W, h, d] as (d, h, b*W) with boxes of 64 x heads x W.
+bool encode_q_beams(CUtensorMap* m, const void* base, int h, int rows, int heads, int beams) {
+  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h), cuuint64_t(rows)};
+  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(h) * kD * 2};
+  const cuuint32_t box[3] = {64, cuuint32_t(heads), cuuint32_t(beams)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_q(CUtensorMap* m, const void* base, int rows, int np) {
   const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(kD) * 2};
@@ -870,7 +891,8 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tk, tv, tq;
   if (!encode_cache(&tk, a.k, a.b, a.m_max, a.g) || !encode_cache(&tv, a.v, a.b, a.m_max, a.g) ||
-      !encode_q(&tq, a.q, a.b * a.h, NP))
+      !(a.q_beams > 0 ? encode_q_beams(&tq, a.q, a.h, a.b * a.q_beams, a.q_group_heads, a.q_beams)
+                      : encode_q(&tq, a.q, a.b * a.h, NP)))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(a.grid));

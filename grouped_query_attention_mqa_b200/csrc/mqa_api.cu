@@ -121,6 +121,9 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.d = d_k;
   a.hq = hq;
   a.window = opts ? opts->window : 0;
+  a.q_beams = 0;
+  a.q_group_heads = hq;
+  a.emit_partials = 0;
   // When no sequence spans more than one tile no segment is ever split, so
   // every output row is final when the decode kernel ends: the merge is left out.
   const int span_max = a.window > 0 && a.window < m_max ? a.window : m_max;
@@ -149,6 +152,87 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
                            const mqa_decode_opts_t* opts, cudaStream_t stream) {
   return decode_impl(o, q, k_cache, v_cache, nullptr, nullptr, lens, b, h, g, m_max, d_k, d_v, scale, dtype,
                      workspace, workspace_bytes_given, status_flags, opts, stream);
+}
+
+size_t mqa_decode_beam_workspace_size(int b, int W, int h, int g, int d_v) {
+  if (b < 0 || W < 1 || h < 1 || g < 1 || h % g != 0 || d_v < 1) return 0;
+  const int hq = h / g;
+  return align256(workspace_bytes(b, g, W * hq, d_v)) + workspace_bytes(b * W, g, hq, d_v);
+}
+
+mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const void* prefix_v,
+                             const int32_t* prefix_lens, const void* suffix_k, const void* suffix_v,
+                             const int32_t* suffix_lens, int b, int W, int h, int g, int m_p, int m_s, int d_k,
+                             int d_v, float scale, mqa_dtype_t dtype, void* workspace, size_t workspace_bytes_given,
+                             int32_t* status_flags, cudaStream_t stream) {
+  if (b < 0 || W < 1 || h < 1 || g < 1 || h % g != 0 || m_p < 1 || m_s < 1 || d_k < 1 || d_v < 1 ||
+      !valid_dtype(dtype) || !std::isfinite(scale))
+    return MQA_ERR_INVALID_ARG;
+  if (b == 0) return MQA_OK;
+  if (!o || !q || !prefix_k || !prefix_v || !prefix_lens || !suffix_k || !suffix_v || !suffix_lens || !workspace)
+    return MQA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(q) || !aligned16(prefix_k) || !aligned16(prefix_v) || !aligned16(prefix_lens) ||
+      !aligned16(suffix_k) || !aligned16(suffix_v) || !aligned16(suffix_lens) || !aligned256(workspace))
+    return MQA_ERR_INVALID_ARG;
+  if (int64_t(b) * W * g > (int64_t(1) << 30) || int64_t(b) * m_p * g > (int64_t(1) << 40) ||
+      int64_t(b) * W * m_s * g > (int64_t(1) << 40) || int64_t(b) * W * h >= (int64_t(1) << 31))
+    return MQA_ERR_INVALID_ARG;
+  const int hq = h / g;
+  if (workspace_bytes_given < mqa_decode_beam_workspace_size(b, W, h, g, d_v)) return MQA_ERR_INVALID_ARG;
+  if (dtype != MQA_BF16 || d_k != d_v || !tc_supported(d_k, W * hq)) return MQA_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return MQA_ERR_CUDA;
+  DecodeArgs a;   // the prefix pass: the W beams' heads of a group read the shared prefix together
+  a.o = o;
+  a.q = q;
+  a.k = prefix_k;
+  a.v = prefix_v;
+  a.k_new = nullptr;
+  a.v_new = nullptr;
+  a.lens = prefix_lens;
+  a.b = b;
+  a.h = h;
+  a.g = g;
+  a.m_max = m_p;
+  a.d = d_k;
+  a.hq = W * hq;
+  a.window = 0;
+  a.no_merge = 0;
+  a.q_beams = W;
+  a.q_group_heads = hq;
+  a.emit_partials = 1;
+  a.scale = scale;
+  a.ws = carve_workspace(workspace, b, g, W * hq);
+  a.flags = status_flags;
+  a.grid = sms * tc_ctas_per_sm(W * hq);
+  DecodeArgs s = a;   // the suffix pass: each beam over its own rows
+  s.k = suffix_k;
+  s.v = suffix_v;
+  s.lens = suffix_lens;
+  s.b = b * W;
+  s.m_max = m_s;
+  s.hq = hq;
+  s.q_beams = 0;
+  s.ws = carve_workspace(static_cast<char*>(workspace) + align256(workspace_bytes(b, g, W * hq, d_v)), b * W, g, hq);
+  s.grid = sms * tc_ctas_per_sm(hq);
+  BeamCombineArgs c;
+  c.o = o;
+  c.plens = prefix_lens;
+  c.slens = suffix_lens;
+  c.b = b;
+  c.W = W;
+  c.h = h;
+  c.g = g;
+  c.hq = hq;
+  c.d = d_v;
+  c.m_p = m_p;
+  c.m_s = m_s;
+  c.pre = a.ws;
+  c.suf = s.ws;
+  if (launch_decode_tc(a, stream) != cudaSuccess || launch_decode_tc(s, stream) != cudaSuccess ||
+      launch_beam_combine(c, stream) != cudaSuccess)
+    return MQA_ERR_CUDA;
+  return MQA_OK;
 }
 
 mqa_status_t mqa_prefill(void* o, const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int b,

@@ -26,7 +26,8 @@ def header_symbols():
 def test_header_declares_the_boundary():
     assert header_symbols() == sorted(["mqa_kv_append", "mqa_decode_workspace_size", "mqa_decode",
                                        "mqa_decode_ex", "mqa_decode_append", "mqa_decode_noalloc",
-                                       "mqa_prefill", "mqa_status_string"])
+                                       "mqa_prefill", "mqa_decode_beam", "mqa_decode_beam_workspace_size",
+                                       "mqa_status_string"])
 
 
 def test_library_exports_every_declared_symbol(lib):
