@@ -29,7 +29,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from grouped_query_attention_mqa_b200.workloads import (PREFILL_WORKLOADS, WORKLOADS,  # noqa: E402
+from grouped_query_attention_mqa_b200.workloads import (BEAM_WORKLOADS, PREFILL_WORKLOADS, WORKLOADS,  # noqa: E402
                                                          append_algorithmic_bytes, decode_algorithmic_bytes,
                                                          draw_lens, f32_to_bf16_bits, bf16_bits_to_f32,
                                                          prefill_flops)
@@ -47,7 +47,8 @@ def parse():
     p.add_argument("--steps", type=int, default=20000)
     p.add_argument("--warmup", type=int, default=200)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS))
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                   choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS) + sorted(BEAM_WORKLOADS))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
     p.add_argument("--num-ctas", type=int, default=0)
     p.add_argument("--window", type=int, default=0, help="local attention: attend to the newest W rows (0 = all)")
@@ -615,9 +616,136 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ beams sharing a prefix
+
+BEAM_METRIC = "beam decode (shared prefix) achieved HBM GB/s vs peak; query-tokens/s"
+
+
+def run_beam(args):
+    """mqa_decode_beam: query-tokens/s (b*W per step) and GB/s of algorithmic
+    bytes (each prefix row once).  Beside it, the same step with every beam
+    holding its own copy of the prefix (b*W sequences through mqa_decode)."""
+    import torch
+    from grouped_query_attention_mqa_b200 import binding
+    from grouped_query_attention_mqa_b200.build import LIB, build
+    from grouped_query_attention_mqa_b200.workloads import beam_algorithmic_bytes, beam_device_inputs
+
+    wl = BEAM_WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from oracle import oracle_decode_beam   # test infrastructure: only the CPU legs of the bench run it
+        rng = np.random.default_rng(SEED)
+        b = 2                                    # a bounded sample: two sequences of the workload's shape
+        lp = rng.integers(wl.lp_lo, wl.lp_hi + 1, size=b)
+        ls = rng.integers(wl.ls_lo, wl.ls_hi + 1, size=b * wl.W)
+        arr = {n: rng.standard_normal(sh, dtype=np.float32) for n, sh in (
+            ("q", (b, wl.W, wl.h, wl.d)), ("pk", (b, wl.m_p, wl.g, wl.d)), ("pv", (b, wl.m_p, wl.g, wl.d)),
+            ("sk", (b * wl.W, wl.m_s, wl.g, wl.d)), ("sv", (b * wl.W, wl.m_s, wl.g, wl.d)))}
+        rates = []
+        for _ in range(max(1, args.steps)):
+            t0 = time.perf_counter()
+            oracle_decode_beam(arr["q"], arr["pk"], arr["pv"], lp, arr["sk"], arr["sv"], ls, wl.g, wl.scale)
+            rates.append(b * wl.W / (time.perf_counter() - t0))
+        value = float(np.median(rates))
+        print(json.dumps({"impl": "reference", "metric": BEAM_METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "config": {"workload": wl.name}, "data": "synthetic",
+                          "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                           "sample": f"2 sequences x {wl.W} beams of {wl.name}, NumPy float64"},
+                          "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    if not os.path.exists(LIB):
+        build()
+    binding.load_library()
+    inp = beam_device_inputs(wl, SEED, "cuda")
+    lp, ls = torch.from_numpy(inp["lp"]).cuda(), torch.from_numpy(inp["ls"]).cuda()
+    out = torch.empty((wl.b, wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(binding.lib().mqa_decode_beam_workspace_size(wl.b, wl.W, wl.h, wl.g, wl.d), dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        binding.decode_beam(inp["q"], inp["pk"], inp["pv"], lp, inp["sk"], inp["sv"], ls, wl.scale, out=out,
+                            workspace=ws)
+
+    def timed(fn, K):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(K):
+            fn()
+        s1.record()
+        torch.cuda.synchronize()
+        return s0.elapsed_time(s1) / K
+
+    K = args.steps
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.2)
+    ms = timed(step, K)
+    clk = clocks.stop()
+    # the same step with the prefix copied into every beam's cache (b*W independent sequences)
+    rows = wl.m_p + wl.m_s
+    rk = torch.zeros((wl.b * wl.W, rows, wl.g, wl.d), dtype=torch.bfloat16, device="cuda")
+    rv = torch.zeros_like(rk)
+    for s_ in range(wl.b):
+        for w in range(wl.W):
+            r, a, c = s_ * wl.W + w, int(inp["lp"][s_]), int(inp["ls"][s_ * wl.W + w])
+            rk[r, :a] = inp["pk"][s_, :a]
+            rv[r, :a] = inp["pv"][s_, :a]
+            rk[r, a:a + c] = inp["sk"][r, :c]
+            rv[r, a:a + c] = inp["sv"][r, :c]
+    rlens = (lp.repeat_interleave(wl.W) + ls).to(torch.int32)
+    rout = torch.empty((wl.b * wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
+    rplan = binding.DecodePlan(inp["q"].view(wl.b * wl.W, wl.h, wl.d), rk, rv, rlens, wl.scale, out=rout)
+    ms_rep = timed(rplan.run, max(10, K // 4))
+    if not torch.allclose(rout.float(), out.view(wl.b * wl.W, wl.h, wl.d).float(), atol=1.5e-2, rtol=0):
+        raise RuntimeError("the shared-prefix and the replicated step disagree")
+    # end to end: q in from pinned host memory and o out, every step
+    q_h = inp["q"].cpu().pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d = torch.empty_like(inp["q"])
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        binding.decode_beam(q_d, inp["pk"], inp["pv"], lp, inp["sk"], inp["sv"], ls, wl.scale, out=out, workspace=ws)
+        o_h.copy_(out, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, max(10, K // 4))
+    alg = beam_algorithmic_bytes(wl, inp["lp"], inp["ls"])
+    peak, peak_kind = peaks()
+    achieved = alg / (ms / 1e3) / 1e9
+    tok = wl.b * wl.W
+    print(json.dumps({
+        "metric": BEAM_METRIC, "value": tok / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "b": wl.b, "beams": wl.W, "h": wl.h, "g": wl.g, "d": wl.d,
+                   "prefix_lens": f"U[{wl.lp_lo},{wl.lp_hi}]", "suffix_lens": f"U[{wl.ls_lo},{wl.ls_hi}]",
+                   "replicated_prefix_ms_per_step": ms_rep,
+                   "replicated_prefix_query_tokens_per_s": tok / (ms_rep / 1e3),
+                   "l2": "the prefix caches exceed the L2 (%d MiB)" % (inp["pk"].numel() * 4 // 2**20)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "one step = prefix decode + suffix decode + combine", "algorithmic_bytes_per_launch": alg,
+                     "launch_ms": ms},
+        "cpu_baseline": None,
+        "e2e": {"value": tok / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": q_h.numel() * 2,
+                "d2h_bytes_per_step": o_h.numel() * 2, "steps": max(10, K // 4)},
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+    }), flush=True)
+
+
 def main():
     args = parse()
-    if args.workload in PREFILL_WORKLOADS:
+    if args.workload in BEAM_WORKLOADS:
+        run_beam(args)
+    elif args.workload in PREFILL_WORKLOADS:
         run_prefill(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -271,3 +271,57 @@ def prefill_device_inputs(wl: PrefillWorkload, seed: int, device):
         out[name] = torch.randn((T, heads, wl.d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
     out["cu"] = torch.arange(0, T + 1, wl.n, dtype=torch.int32, device=device)
     return out
+
+
+@dataclass(frozen=True)
+class BeamWorkload:
+    """One decode step of W beams per sequence sharing a prefix: b sequences,
+    prefix lengths U[lp_lo, lp_hi] (cache m_p rows), suffix lengths
+    U[ls_lo, ls_hi] per beam (cache m_s rows)."""
+    name: str
+    b: int
+    W: int
+    h: int
+    g: int
+    d: int
+    m_p: int
+    lp_lo: int
+    lp_hi: int
+    m_s: int
+    ls_lo: int
+    ls_hi: int
+    scale: float
+    description: str = ""
+
+
+BEAM_WORKLOADS = {
+    "beam4_mqa_b64_p8k": BeamWorkload(
+        "beam4_mqa_b64_p8k", b=64, W=4, h=8, g=1, d=128, m_p=8192, lp_lo=4096, lp_hi=8192, m_s=128, ls_lo=1,
+        ls_hi=128, scale=_S128,
+        description="beam-4 MQA decoder (the paper's h=8, d=128): 64 sequences x 4 beams, prefixes U[4096,8192], "
+                    "suffixes U[1,128]"),
+}
+
+
+def beam_device_inputs(wl: BeamWorkload, seed: int, device):
+    """q [b,W,h,d], prefix caches [b,m_p,g,d], suffix caches [b*W,m_s,g,d] (bf16
+    N(0,1), torch's seeded generator) and the two length arrays (int32)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lp = rng.integers(wl.lp_lo, wl.lp_hi + 1, size=wl.b).astype(np.int32)
+    ls = rng.integers(wl.ls_lo, wl.ls_hi + 1, size=wl.b * wl.W).astype(np.int32)
+
+    def rnd(shape):
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    return {"q": rnd((wl.b, wl.W, wl.h, wl.d)), "pk": rnd((wl.b, wl.m_p, wl.g, wl.d)),
+            "pv": rnd((wl.b, wl.m_p, wl.g, wl.d)), "sk": rnd((wl.b * wl.W, wl.m_s, wl.g, wl.d)),
+            "sv": rnd((wl.b * wl.W, wl.m_s, wl.g, wl.d)), "lp": lp, "ls": ls}
+
+
+def beam_algorithmic_bytes(wl: BeamWorkload, lp, ls) -> int:
+    """Every prefix row once (shared by the beams), every suffix row once, q and o."""
+    rows = int(np.asarray(lp, dtype=np.int64).sum() + np.asarray(ls, dtype=np.int64).sum())
+    return rows * wl.g * 2 * wl.d * 2 + wl.b * wl.W * wl.h * 2 * wl.d * 2
