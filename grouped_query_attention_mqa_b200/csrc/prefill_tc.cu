@@ -327,8 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x2 = 0; x2 < 4; ++x2) {
           const float e0 = ex2_approx(s[ch * 8 + 2 * x2] - m_ref);
           const float e1 = ex2_approx(s[ch * 8 + 2 * x2 + 1] - m_ref);
-          l += e0 + e1;
           __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+          const float2 rounded = __bfloat1622float2(b2);   // the sum uses the P the product sees
+          l += rounded.x + rounded.y;
           packed[x2] = *reinterpret_cast<uint32_t*>(&b2);
         }
         const int half = ch >> 3, c16 = ch & 7;
