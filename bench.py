@@ -295,23 +295,32 @@ def run_ours(args):
     lens = torch.from_numpy(lens_np).cuda()
     out = torch.empty((b, h, wl.d_v), dtype=inp["q"].dtype, device="cuda")
     ws = binding.new_workspace(b, h, g, wl.d_v)
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream()   # the steps' stream; their launches are captured in CUDA graphs
     # one pre-marshalled fused step (append at row lens-1, then decode) per cache copy
     steps = [binding.DecodePlan(inp["q"], inp["k"][c], inp["v"][c], lens, wl.scale, out=out, workspace=ws,
-                                window=args.window,
-                                path=path, num_ctas=args.num_ctas, k_new=inp["k_new"], v_new=inp["v_new"])
+                                window=args.window, path=path, num_ctas=args.num_ctas, stream=stream,
+                                k_new=inp["k_new"], v_new=inp["v_new"])
              for c in range(copies)]
 
-    def step(i):
-        steps[i % copies].run()
-
-    for i in range(max(3, args.warmup)):
-        step(i)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            steps[i % copies].run()
+    torch.cuda.synchronize()
+    # A serving loop replays its steps from a CUDA graph: G steps per graph (a
+    # multiple of the cache copies, so the rotation runs on across replays).
+    G_dev = 40 * copies
+    dev_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(dev_graph, stream=stream):
+        for i in range(G_dev):
+            steps[i % copies].run()
+    with torch.cuda.stream(stream):
+        dev_graph.replay()
     torch.cuda.synchronize()
 
-    # timed region: K steps back to back, CUDA events on the launching stream
-    # around the whole run (events between steps would break the programmatic
-    # dependent launch between one step's merge and the next step's decode)
+    # timed region: exactly K steps back to back (K // G graph replays, the
+    # rest launched one by one), CUDA events on the steps' stream around the
+    # whole run (events between steps would break the programmatic dependent
+    # launch between one step's merge and the next step's decode)
     K = args.steps
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -319,10 +328,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     time.sleep(0.2)
-    start.record(stream)
-    for i in range(K):
-        steps[i % copies].run()
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(K // G_dev):
+            dev_graph.replay()
+        for i in range(K - K % G_dev, K):
+            steps[i % copies].run()
+        end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
@@ -412,10 +424,11 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(R):
-        graph.replay()
-    e2.record(stream)
+    with torch.cuda.stream(stream):   # the replays and the events that bracket them share one stream
+        s2.record(stream)
+        for _ in range(R):
+            graph.replay()
+        e2.record(stream)
     torch.cuda.synchronize()
     # same inputs and a deterministic partition: the last pipelined output equals the device-resident
     # step's on the same cache copy
@@ -449,6 +462,7 @@ def run_ours(args):
                        "l2": f"{copies} rotating K/V cache copies ({copies * cache_bytes / 2**20:.0f} MiB) so each "
                              f"step's rows were evicted by >= 2 other steps' reads",
                        "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)",
+                       "launch": f"CUDA graphs of {G_dev} steps replayed back to back",
                        **({"window": args.window} if args.window else {})},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "peak_kind": peak_kind,
