@@ -20,7 +20,18 @@
 // at row lens-1 and then loads the tile, so the row is both stored for later
 // steps and attended to now.
 //
-// Roles (one CTA per SM, persistent over an even share of all tiles):
+// Work: one CTA per SM, persistent over a contiguous run of all segments'
+// tiles; runs are balanced in quarter tiles with a segment's entry weighted
+// as half a tile.  The thread of the schedule that finds a CTA's first tile
+// issues its first Q, K and V loads itself (start-up code runs at
+// instruction-fetch speed; a separate role would reach them much later).
+// A segment split between CTAs leaves normalised partials with their
+// log-sum-exp for the merge kernel; a whole one is written directly.  With a
+// local window the partition counts only the window's rows.  Beams sharing a
+// prefix: with q_beams the W beams' heads of a group form the segment's query
+// rows (a 3-D box gathers them), and every segment leaves a partial.
+//
+// Roles:
 //   warp 0, lane 0      TMA producer of Q (per segment) and of K tiles into a
 //                       ring of SK stages; a K stage is released as soon as
 //                       the S product that reads it has completed.
@@ -35,12 +46,14 @@
 //                       tcgen05.commit on mbarriers.
 //   warps 2-9           softmax and epilogue in two column groups of four
 //                       warps: one cache row (then one output column) and
-//                       half of the heads per thread.  The reference max per head is set
-//                       from the first tile of a segment and only moved when
-//                       some logit exceeds it by more than 8 (a factor 256 in
-//                       exp2); only then do the warps reduce column maxima and
-//                       rescale O in tensor memory.  P = exp2(s - m) goes to
-//                       shared memory in bf16, per-head sums stay in registers.
+//                       half of the heads per thread.  The reference max per
+//                       head is set from the first tile of a segment and only
+//                       moved when some logit exceeds it by more than 8 (a
+//                       factor 256 in exp2); only then do the warps reduce
+//                       column maxima and rescale O in tensor memory.
+//                       P = exp2(s - m) goes to shared memory in bf16, per-head
+//                       sums stay in registers; a finished segment's O is
+//                       stored straight from the tensor-memory registers.
 // Every wait is bounded (one second); on expiry the kernel sets
 // MQA_FLAG_PIPE_TIMEOUT, drains its own copies and MMAs, frees its tensor
 // memory and returns.
