@@ -229,11 +229,16 @@ def peaks():
 
 
 def source_digest(path_name):
+    """Digest of the kernel sources behind a recorded ncu traffic figure: the
+    code only (comments and blank lines dropped), so a comment edit keeps it."""
     files = ["common.cuh", "decode_tc.cu" if path_name == "tcgen05" else "decode_simt.cu", "merge.cu"]
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "grouped_query_attention_mqa_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "grouped_query_attention_mqa_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
