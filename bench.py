@@ -750,7 +750,8 @@ def run_beam(args):
                    "l2": "the prefix caches exceed the L2 (%d MiB)" % (inp["pk"].numel() * 4 // 2**20)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "one step = prefix decode + suffix decode + combine", "algorithmic_bytes_per_launch": alg,
+                     "kernel": "one step = decode_tc_beam_kernel (prefix once for the W beams, then each beam's "
+                               "suffix) + merge_kernel", "algorithmic_bytes_per_launch": alg,
                      "launch_ms": ms},
         "cpu_baseline": None,
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": q_h.numel() * 2,

@@ -112,6 +112,23 @@ __device__ __forceinline__ int tiles_of(int len, int tile) { return (len + tile 
 // tile k of a segment starts at cache row (len - span) + k * tile.
 __device__ __forceinline__ int span_of(int len, int window) { return window > 0 && len > window ? window : len; }
 
+// Beams sharing a prefix in one pass: sequence s owns, after its prefix rows,
+// the suffix rows of its W beams (beam w's cache row block is s*W + w), each
+// beam's rows starting at a tile edge.  slens == nullptr: no suffixes.
+struct BeamSuffixes {
+  const int32_t* slens;   // [b*W] suffix lengths (clamped to [0, m_s])
+  int W;
+  int m_s;
+};
+
+__device__ __forceinline__ int suffix_tiles(const BeamSuffixes& bs, int s, int tile, int32_t* flags, bool report) {
+  if (bs.slens == nullptr) return 0;
+  int n = 0;
+  for (int w = 0; w < bs.W; ++w)
+    n += tiles_of(clamp_len(__ldg(bs.slens + int64_t(s) * bs.W + w), bs.m_s, flags, report), tile);
+  return n;
+}
+
 __device__ __forceinline__ int64_t range_start(int64_t c, int64_t total, int active) {
   return (c * total) / active;
 }
@@ -210,14 +227,16 @@ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t wtotal, int active
 
 template <int NT>
 __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b, int g, int m_max, int window,
-                                         int tile, int grid, int cta, int32_t* flags, int64_t* red, int xw) {
+                                         int tile, int grid, int cta, int32_t* flags, int64_t* red, int xw,
+                                         const BeamSuffixes& bs) {
   static_assert(NT % 32 == 0, "whole warps");
   const int per = (b + NT - 1) / NT;
   const int s0 = min(b, int(threadIdx.x) * per);
   const int s1 = min(b, s0 + per);
   int64_t my_t = 0, my_u = 0;
   for (int s = s0; s < s1; ++s) {
-    const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), window), tile);
+    const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, flags, cta == 0), window), tile) +
+                   suffix_tiles(bs, s, tile, flags, cta == 0);
     my_t += int64_t(g) * nb;
     my_u += seq_units(nb, g, xw);
   }
@@ -272,7 +291,8 @@ __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b
     if (!(u >= excl_u && u < excl_u + my_u)) return;
     int64_t tb = excl_t, ub = excl_u;
     for (int s = s0; s < s1; ++s) {
-      const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), window), tile);
+      const int nb = tiles_of(span_of(clamp_len(__ldg(lens + s), m_max, nullptr, false), window), tile) +
+                     suffix_tiles(bs, s, tile, nullptr, false);
       const int64_t su = seq_units(nb, g, xw);
       if (u < ub + su) {
         const int64_t seglen = xw + 4 * int64_t(nb);
@@ -315,22 +335,25 @@ __device__ WSched make_schedule_weighted(const int32_t* __restrict__ lens, int b
 // has started to load (WSched::pre).  Code that runs once per launch executes
 // at instruction-fetch speed, so this gets the first loads out well before a
 // separate role would reach them.
-__device__ __forceinline__ bool small_schedule_fits(int b, int g, int m_max, int tile, int nt, int xw) {
-  return b <= nt && int64_t(b) * g * (xw + 4 * (int64_t(m_max) + tile - 1) / tile) < (int64_t(1) << 31);
+__device__ __forceinline__ bool small_schedule_fits(int b, int g, int m_max, int tile, int nt, int xw,
+                                                    int64_t suffix_tiles_max = 0) {
+  return b <= nt && int64_t(b) * g * (xw + 4 * ((int64_t(m_max) + tile - 1) / tile + suffix_tiles_max)) <
+                        (int64_t(1) << 31);
 }
 
 template <int NT, typename OnFirst>
 __device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, int g, int m_max, int window, int tile,
                                       int grid, int cta, int32_t* flags, int64_t* red, int xw, int* lens_tab,
-                                      OnFirst&& on_first) {
+                                      const BeamSuffixes& bs, OnFirst&& on_first) {
   static_assert(NT % 32 == 0, "whole warps");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int len = 0;
+  int len = 0, nsuf = 0;
   if (tid < b) {
     len = clamp_len(__ldg(lens + tid), m_max, flags, cta == 0);
     lens_tab[tid] = len;
+    nsuf = suffix_tiles(bs, tid, tile, flags, cta == 0);
   }
-  const int nb = tiles_of(span_of(len, window), tile);
+  const int nb = tiles_of(span_of(len, window), tile) + nsuf;
   const int my_t = g * nb;
   const int my_u = nb > 0 ? g * (xw + 4 * nb) : 0;
   uint64_t x = (uint64_t(uint32_t(my_t)) << 32) | uint32_t(my_u);
@@ -436,6 +459,8 @@ __device__ __forceinline__ void cursor_seek(Cursor& cu, const int32_t* __restric
 struct TileCoord {
   int seq, head, k;   // sequence, K/V head, tile index within the segment
   int row0, rows;     // first cache row and number of valid rows in the tile
+  int beam;           // beams sharing a prefix: the beam whose suffix the tile is, -1 for a prefix tile
+  int src_row;        // row of the tile's first row in its cache viewed as (rows, g, d)
   int64_t seg;        // segment number seq*g + head
   int64_t seg_t0;     // global number of the segment's first tile
   int nb;             // tiles in the segment
@@ -475,11 +500,18 @@ struct DecodeArgs {
   int q_beams;         // 0: q is [b, h, d]; W > 0: q is [b, W, h, d] and a segment's query rows
                        // are the W beams' q_group_heads heads of its group (hq = W * q_group_heads)
   int q_group_heads;   // query heads per K/V head in q
-  int emit_partials;   // every segment leaves a partial and seg_info; o is not written
   float scale;
   Workspace ws;
   int32_t* flags;
   int grid;
+  // Beams sharing a prefix in one pass (q_beams = W > 0 and sk != nullptr): segment (b, j) walks
+  // sequence b's prefix rows (k, v, lens, m_max), then each beam's own suffix rows (sk, sv,
+  // slens [b*W], m_s; beam w's rows at cache row block b*W + w).  A suffix tile of beam w counts
+  // for that beam's q_group_heads query columns only; o is [b, W, h, d].
+  const void* sk;
+  const void* sv;
+  const int32_t* slens;
+  int m_s;
 };
 
 cudaError_t launch_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos,
@@ -489,14 +521,6 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStrea
 int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq);
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
-struct BeamCombineArgs {
-  void* o;                    // [b, W, h, d] bf16
-  const int32_t* plens;       // [b] prefix lengths
-  const int32_t* slens;       // [b*W] suffix lengths
-  int b, W, h, g, hq, d, m_p, m_s;
-  Workspace pre, suf;         // partials of the prefix and the suffix pass
-};
-cudaError_t launch_beam_combine(const BeamCombineArgs& c, cudaStream_t stream);
 bool prefill_tc_supported(int d, int hq);
 cudaError_t launch_prefill_tc(void* o, const void* q, const void* k, const void* v, const int32_t* cu, int b,
                               int64_t total, int h, int g, int max_seqlen, float scale, int causal, int32_t* flags,

@@ -121,8 +121,11 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.window = 0;
   a.q_beams = 0;
   a.q_group_heads = hq;
-  a.emit_partials = 0;
   a.no_merge = 0;
+  a.sk = nullptr;
+  a.sv = nullptr;
+  a.slens = nullptr;
+  a.m_s = 0;
   a.scale = scale;
   a.ws = carve(scratch, b, g, hq, segs + size_t(grid));
   a.flags = status_flags;

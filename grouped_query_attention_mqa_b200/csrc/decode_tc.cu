@@ -199,16 +199,59 @@ __device__ __forceinline__ bool wait_bar(const Roles& r, uint32_t bar, uint32_t 
   return false;
 }
 
+// Beams sharing a prefix in one pass: the suffixes of the segment's sequence.
+__device__ __forceinline__ BeamSuffixes beam_suffixes(const DecodeArgs& a) {
+  BeamSuffixes bs;
+  bs.slens = a.slens;
+  bs.W = a.q_beams;
+  bs.m_s = a.m_s;
+  return bs;
+}
+
+// Cache rows of tile k of sequence seq: tile k of its attended span (k < nbp),
+// or, with beams sharing a prefix (kFB), a tile of one beam's suffix, the
+// beams' suffixes following the prefix in beam order.
+template <bool kFB>
+__device__ __forceinline__ void locate_tile(const DecodeArgs& a, int seq, int k, int len, int lo, int nbp,
+                                            TileCoord& tc) {
+  if (!kFB || k < nbp) {
+    tc.beam = -1;
+    tc.row0 = lo + k * kTile;
+    tc.rows = min(kTile, len - tc.row0);
+    tc.src_row = seq * a.m_max + tc.row0;
+    return;
+  }
+  int kk = k - nbp;
+  for (int w = 0; w < a.q_beams; ++w) {
+    const int ls = clamp_len(__ldg(a.slens + seq * a.q_beams + w), a.m_s, nullptr, false);
+    const int t = tiles_of(ls, kTile);
+    if (kk < t) {
+      tc.beam = w;
+      tc.row0 = kk * kTile;
+      tc.rows = min(kTile, ls - tc.row0);
+      tc.src_row = (seq * a.q_beams + w) * a.m_s + tc.row0;
+      return;
+    }
+    kk -= t;
+  }
+  tc.beam = 0;   // k beyond the segment: not reached
+  tc.row0 = 0;
+  tc.rows = 0;
+  tc.src_row = 0;
+}
+
 // Walks the CTA's tiles in order and tells each role what a tile is.  Only
 // the first step divides; later steps count (tile, head, sequence) forward.
 // It also tracks the partition units, so that the owner of any tile can be
 // computed.
+template <bool kFB>
 struct TileWalk {
   int64_t t;                 // current tile number
   int64_t base;              // first tile of the current sequence
   int64_t ubase;             // first partition unit of the current sequence
   int seq, head, k, nb, len;
   int lo;                    // first attended row of the sequence (len - span)
+  int nbp;                   // tiles of the attended span (the prefix, with beams)
   int sidx;                  // segment number within this CTA
   TileCoord tc;
   bool first, last;
@@ -232,6 +275,10 @@ struct TileWalk {
     len = seq_len(a, r, s);
     lo = len - span_of(len, a.window);
     nb = tiles_of(len - lo, kTile);
+    if constexpr (kFB) {
+      nbp = nb;
+      nb += suffix_tiles(beam_suffixes(a), s, kTile, nullptr, false);
+    }
   }
   __device__ void next(const DecodeArgs& a, const Sched& sc) {
     ++t;
@@ -249,8 +296,12 @@ struct TileWalk {
     tc.seq = seq;
     tc.head = head;
     tc.k = k;
-    tc.row0 = lo + k * kTile;
-    tc.rows = min(kTile, len - tc.row0);
+    if constexpr (kFB) {
+      locate_tile<kFB>(a, seq, k, len, lo, nbp, tc);
+    } else {
+      tc.row0 = lo + k * kTile;
+      tc.rows = min(kTile, len - tc.row0);
+    }
     tc.seg = int64_t(seq) * a.g + head;
     tc.nb = nb;
     tc.seg_t0 = base + int64_t(head) * nb;
@@ -302,9 +353,10 @@ __device__ __forceinline__ void append_new_row(const DecodeArgs& a, bool is_k, i
 // them: Q of the segment into Q buffer 0 and the first min(2, own) K and V
 // tiles into stages 0 and 1 (K before V, as the producers order them).
 // Returns the number of tiles started; the producers skip those.
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, bool kFB>
 __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const CUtensorMap* tm_q, int seq, int head, int k0, int own, int len, int nb) {
+                         const CUtensorMap* tm_q, const CUtensorMap* tm_sk, const CUtensorMap* tm_sv, int seq,
+                         int head, int k0, int own, int len, int nb) {
   using C = TcCfg<NP, SK, SV>;
   static_assert(SK >= 2 && SV >= 2, "two stages of each ring");
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
@@ -317,24 +369,37 @@ __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap*
       append_new_row(a, true, seq, head, len);
       append_new_row(a, false, seq, head, len);
     }
-    const int row0 = len - span_of(len, a.window) + k * kTile;
-    const int row = seq * a.m_max + row0;
+    int row;
+    const CUtensorMap* mk = tm_k;
+    const CUtensorMap* mv = tm_v;
+    if constexpr (kFB) {
+      const int lo = len - span_of(len, a.window);
+      TileCoord tc;
+      locate_tile<kFB>(a, seq, k, len, lo, tiles_of(len - lo, kTile), tc);
+      row = tc.src_row;
+      if (tc.beam >= 0) {
+        mk = tm_sk;
+        mv = tm_sv;
+      }
+    } else {
+      row = seq * a.m_max + len - span_of(len, a.window) + k * kTile;
+    }
     const uint32_t kdst = r.sbase + C::kK + i * kTileBytes;
     mbar_expect_tx(bar(C::kKFull + i), kTileBytes);
-    tma_load_3d(kdst, tm_k, bar(C::kKFull + i), 0, head, row, pol);
-    tma_load_3d(kdst + kHalfBytes, tm_k, bar(C::kKFull + i), 64, head, row, pol);
+    tma_load_3d(kdst, mk, bar(C::kKFull + i), 0, head, row, pol);
+    tma_load_3d(kdst + kHalfBytes, mk, bar(C::kKFull + i), 64, head, row, pol);
     const uint32_t vdst = r.sbase + C::kV + i * kTileBytes;
     mbar_expect_tx(bar(C::kVFull + i), kTileBytes);
-    tma_load_3d(vdst, tm_v, bar(C::kVFull + i), 0, head, row, pol);
-    tma_load_3d(vdst + kHalfBytes, tm_v, bar(C::kVFull + i), 64, head, row, pol);
+    tma_load_3d(vdst, mv, bar(C::kVFull + i), 0, head, row, pol);
+    tma_load_3d(vdst + kHalfBytes, mv, bar(C::kVFull + i), 64, head, row, pol);
   }
   return npre;
 }
 
 // K ring and the per-segment Q (kIsK), or the V ring.
-template <int NP, int SK, int SV, bool kIsK>
+template <int NP, int SK, int SV, bool kIsK, bool kFB>
 __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, const CUtensorMap* tm_kv,
-                         const CUtensorMap* tm_q) {
+                         const CUtensorMap* tm_q, const CUtensorMap* tm_skv) {
   using C = TcCfg<NP, SK, SV>;
   const Sched& sc = ws.s;
   constexpr int S = kIsK ? SK : SV;
@@ -343,7 +408,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
   constexpr uint32_t kRing = kIsK ? C::kK : C::kV;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  TileWalk w(a, ws, r);
+  TileWalk<kFB> w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t i = 0;
   int q_issued = -1;
@@ -373,13 +438,20 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
         if ((++polls & 1023u) == 0 && polls > (1u << 24)) break;   // cannot stall for good: K gives up on abort
       }
     }
-    const int row = w.tc.seq * a.m_max + w.tc.row0;
+    int row;
+    const CUtensorMap* map = tm_kv;
+    if constexpr (kFB) {
+      row = w.tc.src_row;
+      if (w.tc.beam >= 0) map = tm_skv;
+    } else {
+      row = w.tc.seq * a.m_max + w.tc.row0;
+    }
     const uint32_t dst = r.sbase + kRing + st * kTileBytes;
     if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1)   // this tile holds the sequence's newest row
       append_new_row(a, kIsK, w.tc.seq, w.tc.head, w.len);
     mbar_expect_tx(bar(kFull + st), kTileBytes);
-    tma_load_3d(dst, tm_kv, bar(kFull + st), 0, w.tc.head, row, pol);
-    tma_load_3d(dst + kHalfBytes, tm_kv, bar(kFull + st), 64, w.tc.head, row, pol);
+    tma_load_3d(dst, map, bar(kFull + st), 0, w.tc.head, row, pol);
+    tma_load_3d(dst + kHalfBytes, map, bar(kFull + st), 64, w.tc.head, row, pol);
     if (kIsK) *reinterpret_cast<volatile int*>(r.smem + C::kKIssued) = int(i + 1);
   }
   // Drain: every copy this thread issued has landed before the CTA can exit.
@@ -396,7 +468,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
 // V(j) has landed.  The two streams are independent, so the thread polls both
 // and issues whichever is ready: a late K tile never holds up a P.V product
 // the softmax warps are waiting for.
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, bool kFB>
 __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
   using C = TcCfg<NP, SK, SV>;
   const Sched& sc = ws.s;
@@ -404,7 +476,7 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int64_t n = sc.t_end - sc.t_begin;
-  TileWalk wq(a, ws, r), wp(a, ws, r);   // walkers for the S stream and the O stream
+  TileWalk<kFB> wq(a, ws, r), wp(a, ws, r);   // walkers for the S stream and the O stream
   const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);           // K-major, rows of 128 B
   const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
   const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
@@ -487,7 +559,7 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
   mbar_wait(bar(C::kDone), 0, kTimeoutNs);
 }
 
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, bool kFB>
 __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Roles& r, int warp, int lane) {
   using C = TcCfg<NP, SK, SV>;
   const Sched& sc = ws.s;
@@ -518,7 +590,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     for (int k = tid; k < int(C::kPBytes / 16); k += 256) p[k] = make_uint4(0, 0, 0, 0);
     named_barrier_softmax();
   }
-  TileWalk w(a, ws, r);
+  TileWalk<kFB> w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t pv_waited = -1;
   bool failed = false;
@@ -543,12 +615,27 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     const int64_t slot = partial_slot(blockIdx.x, e.seg);
     float v[CPT];
     tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
-    if (e.whole && !a.emit_partials) {
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) +
-                           (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * kD + row;
+    if (e.whole) {
+      if constexpr (kFB) {   // column (w, i) of the segment is head i of the group in beam w's output row
+        const int qgh = a.q_group_heads;
+        int bw = col0 / qgh, bi = col0 - bw * qgh;
 #pragma unroll
-      for (int k = 0; k < CPT; ++k)
-        if (col0 + k < hq) dst[k * kD] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+        for (int k = 0; k < CPT; ++k) {
+          if (col0 + k < hq)
+            static_cast<__nv_bfloat16*>(a.o)[((int64_t(e.seq) * a.q_beams + bw) * a.h + int64_t(e.head) * qgh + bi) *
+                                                 kD + row] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+          if (++bi == qgh) {
+            bi = 0;
+            ++bw;
+          }
+        }
+      } else {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) +
+                             (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * kD + row;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+          if (col0 + k < hq) dst[k * kD] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+      }
     } else {
       float* dst = a.ws.part_o + (slot * hq + col0) * kD + row;
 #pragma unroll
@@ -556,7 +643,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
         if (col0 + k < hq) dst[k * kD] = v[k] * linv[pb * NP + col0 + k];
     }
     if (warp == 2) {
-      if (!e.whole || a.emit_partials)   // every partial carries its log-sum-exp
+      if (!e.whole)   // every partial carries its log-sum-exp
         for (int col = lane; col < hq; col += 32) a.ws.part_lse[slot * hq + col] = lse2[pb * NP + col];
       if (e.owns_first && lane == 0)
         a.ws.seg_info[e.seg] = make_int2(blockIdx.x, cta_of_unit(e.seg_last_unit, ws.wtotal, sc.active));
@@ -577,6 +664,14 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     tmem_ld<CPT>(t_lane + uint32_t(i & 1) * NP + col0, sv);
 #pragma unroll
     for (int k = 0; k < CPT; ++k) sv[k] = valid ? sv[k] * c : -INFINITY;
+    if constexpr (kFB) {
+      if (w.tc.beam >= 0) {   // a beam's suffix tile counts for that beam's query columns only
+        const int cb0 = w.tc.beam * a.q_group_heads, cb1 = cb0 + a.q_group_heads;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+          if (col0 + k < cb0 || col0 + k >= cb1) sv[k] = -INFINITY;
+      }
+    }
     // Does any logit of a real head exceed the reference max by the threshold?
     bool exceed = false;
     if (!w.first) {
@@ -612,7 +707,9 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
               mn = mo;
             }
           }
-          mref[col] = mn;
+          // With beams a column may have no row yet: a finite floor keeps exp2(s - m) at 0
+          // (s = -inf) instead of NaN, and the first real logit then exceeds it.
+          mref[col] = kFB ? fmaxf(mn, -1e30f) : mn;
           alpha[col] = al;
         }
       }
@@ -702,7 +799,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       if (gw == 0)
         for (int col = col0 + lane; col < col0 + CPT; col += 32) {
           const float l = redl[col] + redl[NP + col] + redl[2 * NP + col] + redl[3 * NP + col];
-          linv[pb * NP + col] = rcp_approx(l);
+          linv[pb * NP + col] = kFB && !(l > 0.f) ? 0.f : rcp_approx(l);   // a beam with no rows here: o = 0
           lse2[pb * NP + col] = mref[col] + lg2_approx(l);
         }
       pend.on = true;
@@ -734,10 +831,10 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 // One CTA per SM.  The warps of a CTA are spread over the SM's four
 // sub-partitions of 16K registers each; with 11 warps three share one, which
 // caps a thread at 168 registers.
-template <int NP, int SK, int SV>
-__global__ void __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
+template <int NP, int SK, int SV, bool kFB>
+__device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                               const CUtensorMap& tm_q, const CUtensorMap& tm_sk,
+                                               const CUtensorMap& tm_sv) {
   using C = TcCfg<NP, SK, SV>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -776,6 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_q);
+    if constexpr (kFB) {
+      prefetch_tensormap(&tm_sk);
+      prefetch_tensormap(&tm_sv);
+    }
   }
   if (warp == 1) {
     tmem_alloc(r.sbase + C::kTmemSlot, kTmemCols);
@@ -788,16 +889,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   r.lens_s = lens_tab;
   int64_t* sched_red = reinterpret_cast<int64_t*>(r.smem + C::kSched);
   WSched ws;
-  if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits)) {
+  BeamSuffixes bs;
+  if constexpr (kFB) {
+    bs = beam_suffixes(a);
+  } else {
+    bs.slens = nullptr;
+    bs.W = 0;
+    bs.m_s = 0;
+  }
+  if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
+                          kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
     ws = make_schedule_small<kThreads>(
-        a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab,
+        a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
         [&](int seq, int head, int k0, int own, int len, int nb) {
-          return pre_issue<NP, SK, SV>(a, r, &tm_k, &tm_v, &tm_q, seq, head, k0, own, len, nb);
+          return pre_issue<NP, SK, SV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, k0, own, len, nb);
         });
     r.seq0 = 0;
   } else {
     ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red,
-                                          kSegUnits);
+                                          kSegUnits, bs);
     r.seq0 = ws.s.seq;
     if (threadIdx.x < kLensCache && ws.s.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them
       lens_tab[threadIdx.x] = clamp_len(__ldg(a.lens + ws.s.seq + threadIdx.x), a.m_max, nullptr, false);
@@ -817,15 +927,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (sc.t_begin < sc.t_end) {
     if (warp == 0) {
-      if (lane == 0) producer<NP, SK, SV, true>(a, ws, r, &tm_k, &tm_q);
+      if (lane == 0) producer<NP, SK, SV, true, kFB>(a, ws, r, &tm_k, &tm_q, &tm_sk);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<NP, SK, SV>(a, ws, r);
+      if (lane == 0) mma_issuer<NP, SK, SV, kFB>(a, ws, r);
     } else if (warp == kVWarp) {
       // V loads from a warp of their own: sharing one with the K loads would
       // serialise the two threads' waits
-      if (lane == 0) producer<NP, SK, SV, false>(a, ws, r, &tm_v, &tm_q);
+      if (lane == 0) producer<NP, SK, SV, false, kFB>(a, ws, r, &tm_v, &tm_q, &tm_sv);
     } else {
-      softmax_epilogue<NP, SK, SV>(a, ws, r, warp, lane);
+      softmax_epilogue<NP, SK, SV, kFB>(a, ws, r, warp, lane);
     }
   }
   tc_fence_before();
@@ -835,6 +945,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The merge kernel may launch now (launching it earlier, to wait beside this
   // grid, measured slower).
   asm volatile("griddepcontrol.launch_dependents;");
+}
+
+template <int NP, int SK, int SV>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
+  decode_tc_body<NP, SK, SV, false>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
+}
+
+// Beams sharing a prefix in one pass: the suffix caches' maps as well.
+template <int NP, int SK, int SV>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_beam_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_sk, const __grid_constant__ CUtensorMap tm_sv) {
+  decode_tc_body<NP, SK, SV, true>(a, tm_k, tm_v, tm_q, tm_sk, tm_sv);
 }
 
 // ------------------------------------------------------------------ host
@@ -889,7 +1015,7 @@ bool encode_q(CUtensorMap* m, const void* base, int rows, int np) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, bool kFB>
 cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   using L = TcCfg<NP, SK, SV>;
   static bool attr_set[64] = {false};
@@ -897,15 +1023,21 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc));
+    e = kFB ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(L::kAlloc))
+            : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(L::kAlloc));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
-  CUtensorMap tk, tv, tq;
+  CUtensorMap tk, tv, tq, tsk, tsv;
   if (!encode_cache(&tk, a.k, a.b, a.m_max, a.g) || !encode_cache(&tv, a.v, a.b, a.m_max, a.g) ||
       !(a.q_beams > 0 ? encode_q_beams(&tq, a.q, a.h, a.b * a.q_beams, a.q_group_heads, a.q_beams)
                       : encode_q(&tq, a.q, a.b * a.h, NP)))
+    return cudaErrorInvalidValue;
+  if (kFB && (!encode_cache(&tsk, a.sk, a.b * a.q_beams, a.m_s, a.g) ||
+              !encode_cache(&tsv, a.sv, a.b * a.q_beams, a.m_s, a.g)))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(a.grid));
@@ -917,6 +1049,7 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV>, a, tk, tv, tq, tsk, tsv);
   return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NP, SK, SV>, a, tk, tv, tq);
 }
 
@@ -931,9 +1064,16 @@ int tc_tile_rows() { return kTile; }
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) || int64_t(a.b) * a.h >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
-  if (a.hq <= 16) return launch_np<16, 2, 3>(a, stream);
-  if (a.hq <= 32) return launch_np<32, 2, 3>(a, stream);
-  if (a.hq <= 64) return launch_np<64, 2, 3>(a, stream);
+  if (a.sk != nullptr) {   // beams sharing a prefix, one pass
+    if (a.q_beams < 1 || int64_t(a.b) * a.q_beams * a.m_s >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    if (a.hq <= 16) return launch_np<16, 2, 3, true>(a, stream);
+    if (a.hq <= 32) return launch_np<32, 2, 3, true>(a, stream);
+    if (a.hq <= 64) return launch_np<64, 2, 3, true>(a, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (a.hq <= 16) return launch_np<16, 2, 3, false>(a, stream);
+  if (a.hq <= 32) return launch_np<32, 2, 3, false>(a, stream);
+  if (a.hq <= 64) return launch_np<64, 2, 3, false>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -123,7 +123,10 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.window = opts ? opts->window : 0;
   a.q_beams = 0;
   a.q_group_heads = hq;
-  a.emit_partials = 0;
+  a.sk = nullptr;
+  a.sv = nullptr;
+  a.slens = nullptr;
+  a.m_s = 0;
   // When no sequence spans more than one tile no segment is ever split, so
   // every output row is final when the decode kernel ends: the merge is left out.
   const int span_max = a.window > 0 && a.window < m_max ? a.window : m_max;
@@ -156,8 +159,7 @@ mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, const vo
 
 size_t mqa_decode_beam_workspace_size(int b, int W, int h, int g, int d_v) {
   if (b < 0 || W < 1 || h < 1 || g < 1 || h % g != 0 || d_v < 1) return 0;
-  const int hq = h / g;
-  return align256(workspace_bytes(b, g, W * hq, d_v)) + workspace_bytes(b * W, g, hq, d_v);
+  return workspace_bytes(b, g, W * (h / g), d_v);
 }
 
 mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const void* prefix_v,
@@ -182,7 +184,10 @@ mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const
   if (dtype != MQA_BF16 || d_k != d_v || !tc_supported(d_k, W * hq)) return MQA_ERR_UNSUPPORTED;
   const int sms = sm_count();
   if (sms <= 0) return MQA_ERR_CUDA;
-  DecodeArgs a;   // the prefix pass: the W beams' heads of a group read the shared prefix together
+  // One pass: segment (s, j) reads sequence s's prefix once for the W beams'
+  // heads of group j (a 3-D box gathers their query rows), then each beam's
+  // suffix rows, which count for that beam's heads only.
+  DecodeArgs a;
   a.o = o;
   a.q = q;
   a.k = prefix_k;
@@ -200,37 +205,15 @@ mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const
   a.no_merge = 0;
   a.q_beams = W;
   a.q_group_heads = hq;
-  a.emit_partials = 1;
+  a.sk = suffix_k;
+  a.sv = suffix_v;
+  a.slens = suffix_lens;
+  a.m_s = m_s;
   a.scale = scale;
   a.ws = carve_workspace(workspace, b, g, W * hq);
   a.flags = status_flags;
   a.grid = sms * tc_ctas_per_sm(W * hq);
-  DecodeArgs s = a;   // the suffix pass: each beam over its own rows
-  s.k = suffix_k;
-  s.v = suffix_v;
-  s.lens = suffix_lens;
-  s.b = b * W;
-  s.m_max = m_s;
-  s.hq = hq;
-  s.q_beams = 0;
-  s.ws = carve_workspace(static_cast<char*>(workspace) + align256(workspace_bytes(b, g, W * hq, d_v)), b * W, g, hq);
-  s.grid = sms * tc_ctas_per_sm(hq);
-  BeamCombineArgs c;
-  c.o = o;
-  c.plens = prefix_lens;
-  c.slens = suffix_lens;
-  c.b = b;
-  c.W = W;
-  c.h = h;
-  c.g = g;
-  c.hq = hq;
-  c.d = d_v;
-  c.m_p = m_p;
-  c.m_s = m_s;
-  c.pre = a.ws;
-  c.suf = s.ws;
-  if (launch_decode_tc(a, stream) != cudaSuccess || launch_decode_tc(s, stream) != cudaSuccess ||
-      launch_beam_combine(c, stream) != cudaSuccess)
+  if (launch_decode_tc(a, stream) != cudaSuccess || launch_merge(a, dtype, stream) != cudaSuccess)
     return MQA_ERR_CUDA;
   return MQA_OK;
 }

@@ -239,10 +239,11 @@ MQA_API mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k_ca
  * a beam-4 decoder (MQA 32 us vs MHA 203 us per token; local MQA 16 us); the
  * pages give no formula.  Reading: beam w of sequence s attends over the
  * prefix rows 0..prefix_lens[s]-1 of sequence s followed by its own suffix
- * rows 0..suffix_lens[s*W+w]-1 (the tokens that beam generated).  The prefix
- * is read once for all W beams: its K/V tiles feed the W beams' query heads of
- * a group together (W*h/g query rows per tile); the suffixes are read per
- * beam; the two parts are combined with their log-sum-exp weights.
+ * rows 0..suffix_lens[s*W+w]-1 (the tokens that beam generated).  One pass:
+ * the prefix is read once for all W beams, its K/V tiles feeding the W beams'
+ * query heads of a group together (W*h/g query rows per tile), and then each
+ * beam's suffix rows, which count for that beam's heads only; sequences split
+ * between CTAs are merged with log-sum-exp weights afterwards.
  *
  *   o            device [b, W, h, d_v]   written
  *   q            device [b, W, h, d_k]
