@@ -229,9 +229,10 @@ def peaks():
 
 
 def source_digest(path_name):
-    """Digest of the kernel sources behind a recorded ncu traffic figure: the
-    code only (comments and blank lines dropped), so a comment edit keeps it."""
-    files = ["common.cuh", "decode_tc.cu" if path_name == "tcgen05" else "decode_simt.cu", "merge.cu"]
+    """Digest of the sources that build the decode kernel behind a recorded
+    ncu traffic figure (the merge kernel is not part of that figure): the code
+    only (comments and blank lines dropped), so a comment edit keeps it."""
+    files = ["common.cuh", "sm100.cuh", "decode_tc.cu" if path_name == "tcgen05" else "decode_simt.cu"]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "grouped_query_attention_mqa_b200", "csrc", f)) as fh:

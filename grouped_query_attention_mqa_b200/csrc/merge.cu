@@ -22,11 +22,20 @@ namespace {
 
 constexpr int kMergeThreads = 128;
 
+// What the merge reads of a decode's arguments (a small parameter block).
+struct MergeArgs {
+  void* o;
+  const int32_t* lens;
+  const int32_t* slens;
+  Workspace ws;
+  int h, g, hq, d, m_max, q_beams, q_group_heads, m_s;
+};
+
 // One CTA per (segment, group of heads); each thread merges four consecutive
 // output columns of one head, so the few partial loads of every output are
 // issued by many threads at once instead of walked serially.
 template <typename T, bool kBeams>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a, int heads_per_cta) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeArgs a, int heads_per_cta) {
   const int hq = a.hq, D = a.d;
   const int chunks = (hq + heads_per_cta - 1) / heads_per_cta;
   const int64_t s = blockIdx.x / chunks;
@@ -115,9 +124,24 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
 
 }  // namespace
 
-cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream) {
+cudaError_t launch_merge(const DecodeArgs& da, mqa_dtype_t dtype, cudaStream_t stream) {
+  MergeArgs a;
+  a.o = da.o;
+  a.lens = da.lens;
+  a.slens = da.slens;
+  a.ws = da.ws;
+  a.h = da.h;
+  a.g = da.g;
+  a.hq = da.hq;
+  a.d = da.d;
+  a.m_max = da.m_max;
+  a.q_beams = da.q_beams;
+  a.q_group_heads = da.q_group_heads;
+  a.m_s = da.m_s;
+  const int b = da.b;
+  const bool beams = da.sk != nullptr;
   const int heads_per_cta = kMergeThreads / (a.d / 4);
-  const int64_t ctas = int64_t(a.b) * a.g * ((a.hq + heads_per_cta - 1) / heads_per_cta);
+  const int64_t ctas = int64_t(b) * a.g * ((a.hq + heads_per_cta - 1) / heads_per_cta);
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(ctas));
@@ -129,7 +153,7 @@ cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.sk != nullptr) return cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16, true>, a, heads_per_cta);
+  if (beams) return cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16, true>, a, heads_per_cta);
   if (dtype == MQA_BF16) return cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16, false>, a, heads_per_cta);
   return cudaLaunchKernelEx(&cfg, merge_kernel<float, false>, a, heads_per_cta);
 }
