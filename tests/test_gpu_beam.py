@@ -86,3 +86,43 @@ def test_beam_shapes_not_built_are_rejected():
     with pytest.raises(binding.MqaError):
         binding.decode_beam(q, pk, pk, torch.ones(1, dtype=torch.int32, device="cuda"), sk, sk,
                             torch.ones(4, dtype=torch.int32, device="cuda"), 1.0)
+
+
+def test_beam_empty_sequences_and_beams():
+    """A sequence with no prefix and no suffix rows in any beam gets zero rows
+    (nothing reads its caches); a sequence with no prefix but suffix rows
+    attends over those only; prefixes long enough to be split between CTAs sit
+    beside them."""
+    b, W, h, g = 4, 4, 8, 1
+    m_p, m_s = 2000, 160
+    lp = np.array([0, 0, 1999, 640], np.int32)
+    ls = np.array([0, 0, 0, 0, 5, 0, 160, 129, 0, 0, 0, 0, 1, 2, 3, 4], np.int32)
+    inp = beam_inputs(b, W, h, g, m_p, m_s, lp, ls, seed=21)
+    o = host64(binding.decode_beam(dev(inp["q"], "bf16"), dev(inp["pk"], "bf16"), dev(inp["pv"], "bf16"),
+                                   torch.from_numpy(lp).cuda(), dev(inp["sk"], "bf16"), dev(inp["sv"], "bf16"),
+                                   torch.from_numpy(ls).cuda(), 1 / math.sqrt(D)))
+    ref, _ = oracle_decode_beam(inp["q_f32"], inp["pk_f32"], inp["pv_f32"], lp, inp["sk_f32"], inp["sv_f32"], ls,
+                                g, 1 / math.sqrt(D))
+    assert_close(o, ref, "bf16", "empty sequences and beams")
+    assert (o[0] == 0).all()           # no rows at all
+    assert (o[1, 1] == 0).all()        # no prefix, empty suffix
+    assert np.isfinite(o).all()
+
+
+def test_beam_suffix_lengths_are_clamped_and_flagged():
+    """Suffix lengths past the suffix cache are clamped to it and reported
+    through the status word; the result is the clamped step's."""
+    b, W, h, g = 2, 2, 16, 2
+    m_p, m_s = 300, 100
+    lp = np.array([300, 17], np.int32)
+    ls_given = np.array([100, 250, -3, 40], np.int32)
+    ls_used = np.clip(ls_given, 0, m_s).astype(np.int32)
+    inp = beam_inputs(b, W, h, g, m_p, m_s, lp, ls_used, seed=22)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = host64(binding.decode_beam(dev(inp["q"], "bf16"), dev(inp["pk"], "bf16"), dev(inp["pv"], "bf16"),
+                                   torch.from_numpy(lp).cuda(), dev(inp["sk"], "bf16"), dev(inp["sv"], "bf16"),
+                                   torch.from_numpy(ls_given).cuda(), 0.2, status_flags=flags))
+    ref, _ = oracle_decode_beam(inp["q_f32"], inp["pk_f32"], inp["pv_f32"], lp, inp["sk_f32"], inp["sv_f32"],
+                                ls_used, g, 0.2)
+    assert_close(o, ref, "bf16", "clamped suffixes")
+    assert int(flags.item()) & binding.MQA_FLAG_LEN_CLAMPED
