@@ -124,7 +124,8 @@ struct BeamSuffixes {
 __device__ __forceinline__ int suffix_tiles(const BeamSuffixes& bs, int s, int tile, int32_t* flags, bool report) {
   if (bs.slens == nullptr) return 0;
   int n = 0;
-  for (int w = 0; w < bs.W; ++w)
+#pragma unroll 4
+  for (int w = 0; w < bs.W; ++w)   // unrolled: the length loads go out together
     n += tiles_of(clamp_len(__ldg(bs.slens + int64_t(s) * bs.W + w), bs.m_s, flags, report), tile);
   return n;
 }
@@ -344,7 +345,7 @@ __device__ __forceinline__ bool small_schedule_fits(int b, int g, int m_max, int
 template <int NT, typename OnFirst>
 __device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, int g, int m_max, int window, int tile,
                                       int grid, int cta, int32_t* flags, int64_t* red, int xw, int* lens_tab,
-                                      const BeamSuffixes& bs, OnFirst&& on_first) {
+                                      const BeamSuffixes& bs, int* nsuf_tab, OnFirst&& on_first) {
   static_assert(NT % 32 == 0, "whole warps");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int len = 0, nsuf = 0;
@@ -352,6 +353,7 @@ __device__ WSched make_schedule_small(const int32_t* __restrict__ lens, int b, i
     len = clamp_len(__ldg(lens + tid), m_max, flags, cta == 0);
     lens_tab[tid] = len;
     nsuf = suffix_tiles(bs, tid, tile, flags, cta == 0);
+    if (nsuf_tab != nullptr) nsuf_tab[tid] = nsuf;
   }
   const int nb = tiles_of(span_of(len, window), tile) + nsuf;
   const int my_t = g * nb;
@@ -474,6 +476,8 @@ __device__ __forceinline__ TileCoord tile_coord(const Cursor& cu, int g, int til
   tc.k = int(rel - int64_t(tc.head) * cu.nb);
   tc.row0 = cu.lo + tc.k * tile;
   tc.rows = min(tile, cu.len - tc.row0);
+  tc.beam = -1;
+  tc.src_row = 0;   // not used by the SIMT path
   tc.seg = int64_t(cu.seq) * g + tc.head;
   tc.nb = cu.nb;
   tc.seg_t0 = cu.base + int64_t(tc.head) * cu.nb;

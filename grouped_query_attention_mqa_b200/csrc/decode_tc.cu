@@ -109,7 +109,8 @@ struct TcCfg {
   static constexpr uint32_t kLens = kLse + 2 * NP * 4;          // [kLensCache] clamped lengths from seq0
   static constexpr uint32_t kKIssued = kLens + kLensCache * 4;   // K tiles issued so far (V producer trails it)
   static constexpr uint32_t kSched = kKIssued + 16;            // start-up scratch of the schedule
-  static constexpr uint32_t kEnd = kSched + 256;
+  static constexpr uint32_t kNsuf = kSched + 256;              // [kLensCache] beams: suffix tiles per sequence
+  static constexpr uint32_t kEnd = kNsuf + kLensCache * 4;
   static constexpr uint32_t kAlloc = kEnd + 1024;             // room to align the base to 1024 bytes
   static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kQBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kAlloc <= kMaxDynSmem, "shared memory budget");
@@ -179,6 +180,7 @@ struct Roles {
   volatile int* abort;
   int32_t* flags;
   const int* lens_s;         // clamped lens[seq0 + i], i < kLensCache (global memory beyond that)
+  const int* nsuf_s;         // beams: suffix tiles of sequence i < kLensCache, or nullptr
   int seq0;                  // 0 when the whole batch is in the table
 };
 
@@ -277,7 +279,8 @@ struct TileWalk {
     nb = tiles_of(len - lo, kTile);
     if constexpr (kFB) {
       nbp = nb;
-      nb += suffix_tiles(beam_suffixes(a), s, kTile, nullptr, false);
+      nb += r.nsuf_s != nullptr && s < kLensCache ? r.nsuf_s[s]
+                                                 : suffix_tiles(beam_suffixes(a), s, kTile, nullptr, false);
     }
   }
   __device__ void next(const DecodeArgs& a, const Sched& sc) {
@@ -887,6 +890,7 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int* lens_tab = reinterpret_cast<int*>(r.smem + C::kLens);
   r.lens_s = lens_tab;
+  r.nsuf_s = nullptr;
   int64_t* sched_red = reinterpret_cast<int64_t*>(r.smem + C::kSched);
   WSched ws;
   BeamSuffixes bs;
@@ -901,10 +905,12 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
                           kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
     ws = make_schedule_small<kThreads>(
         a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
+        kFB ? reinterpret_cast<int*>(r.smem + C::kNsuf) : nullptr,
         [&](int seq, int head, int k0, int own, int len, int nb) {
           return pre_issue<NP, SK, SV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, k0, own, len, nb);
         });
     r.seq0 = 0;
+    if (kFB) r.nsuf_s = reinterpret_cast<const int*>(r.smem + C::kNsuf);
   } else {
     ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red,
                                           kSegUnits, bs);
