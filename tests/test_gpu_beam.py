@@ -126,3 +126,22 @@ def test_beam_suffix_lengths_are_clamped_and_flagged():
                                 ls_used, g, 0.2)
     assert_close(o, ref, "bf16", "clamped suffixes")
     assert int(flags.item()) & binding.MQA_FLAG_LEN_CLAMPED
+
+
+def test_beam_many_sequences_weighted_schedule():
+    """More sequences than the decode CTA has threads (353 > 352): the schedule
+    takes its general path, where the tile walkers count suffix tiles from
+    global memory; results still match the oracle."""
+    b, W, h, g = 353, 2, 8, 1
+    m_p, m_s = 300, 40
+    rng = np.random.default_rng(353)
+    lp = rng.integers(0, m_p + 1, size=b).astype(np.int32)
+    ls = rng.integers(0, m_s + 1, size=b * W).astype(np.int32)
+    inp = beam_inputs(b, W, h, g, m_p, m_s, lp, ls, seed=353)
+    scale = 1 / math.sqrt(D)
+    o = host64(binding.decode_beam(dev(inp["q"], "bf16"), dev(inp["pk"], "bf16"), dev(inp["pv"], "bf16"),
+                                   torch.from_numpy(lp).cuda(), dev(inp["sk"], "bf16"), dev(inp["sv"], "bf16"),
+                                   torch.from_numpy(ls).cuda(), scale))
+    ref, _ = oracle_decode_beam(inp["q_f32"], inp["pk_f32"], inp["pv_f32"], lp, inp["sk_f32"], inp["sv_f32"], ls,
+                                g, scale)
+    assert_close(o, ref, "bf16", "353 sequences")
