@@ -901,33 +901,8 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     bs.W = 0;
     bs.m_s = 0;
   }
-  if (!kFB && a.no_merge && int64_t(a.b) * a.g <= a.grid) {
-    // Every sequence fits one tile and there are no more (sequence, K/V head)
-    // segments than CTAs: CTA c takes segment c whole.  No scan: one length
-    // load, then at once the loads of the segment's Q, K and V.
-    const int c = blockIdx.x, nseg = a.b * a.g;
-    const int seq = c < nseg ? c / a.g : 0, head = c < nseg ? c - seq * a.g : 0;
-    if (threadIdx.x == 0) {
-      const int len = c < nseg ? clamp_len(__ldg(a.lens + seq), a.m_max, a.flags, head == 0) : 0;
-      lens_tab[0] = len;
-      sched_red[0] = len > 0 ? pre_issue<NP, SK, SV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, 0, 1,
-                                                           len, 1)
-                             : 0;
-    }
-    __syncthreads();
-    const bool work = lens_tab[0] > 0;
-    ws.s.total = nseg;
-    ws.s.active = a.grid;
-    ws.s.t_begin = work ? c : 0;   // tile c: segment c's only tile
-    ws.s.t_end = work ? c + 1 : 0;
-    ws.s.seq = seq;
-    ws.s.seq_base = int64_t(seq) * a.g;
-    ws.wtotal = 1;
-    ws.seq_ubase = 0;
-    ws.pre = int(sched_red[0]);
-    r.seq0 = seq;                  // lens_tab[0] holds this sequence's length
-  } else if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
-                                 kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
+  if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
+                          kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
     ws = make_schedule_small<kThreads>(
         a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
         kFB ? reinterpret_cast<int*>(r.smem + C::kNsuf) : nullptr,
