@@ -521,8 +521,9 @@ struct DecodeArgs {
 cudaError_t launch_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos,
                           int b, int m_max, int g, int row_k_bytes, int row_v_bytes, int32_t* flags,
                           cudaStream_t stream);
-cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
-int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq);
+// The CUDA-core decode: q and K rows of d_k elements, V and o rows of a.d = d_v.
+cudaError_t launch_decode_simt(const DecodeArgs& a, int d_k, mqa_dtype_t dtype, cudaStream_t stream);
+int simt_ctas_per_sm(mqa_dtype_t dtype, int d_k, int d_v, int hq);
 cudaError_t launch_merge(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 bool prefill_tc_supported(int d, int hq);

@@ -82,10 +82,10 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
     return MQA_ERR_INVALID_ARG;
   if (int64_t(b) * g > (int64_t(1) << 30) || int64_t(b) * m_max * g > (int64_t(1) << 40))
     return MQA_ERR_INVALID_ARG;
-  if (d_k != d_v || (d_k != 32 && d_k != 64 && d_k != 128)) return MQA_ERR_UNSUPPORTED;
+  if ((d_k != 32 && d_k != 64 && d_k != 128) || (d_v != 32 && d_v != 64 && d_v != 128)) return MQA_ERR_UNSUPPORTED;
   const int hq = h / g;
-  const bool use_tc = dtype == MQA_BF16 && tc_supported(d_k, hq) && hq >= 8;
-  if (!use_tc && int64_t(hq) * d_k > 4096) return MQA_ERR_UNSUPPORTED;
+  const bool use_tc = dtype == MQA_BF16 && d_k == d_v && tc_supported(d_k, hq) && hq >= 8;
+  if (!use_tc && (int64_t(hq) * d_k > 4096 || int64_t(hq) * d_v > 4096)) return MQA_ERR_UNSUPPORTED;
 
   // Largest CTA count whose partials fit the array; reject when even one CTA
   // does not fit.
@@ -93,7 +93,7 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   if (scratch_bytes(b, g, hq, d_v, segs + 1) > size_t(MQA_NOALLOC_SCRATCH_BYTES)) return MQA_ERR_INVALID_ARG;
   const int sms = sm_count_current();
   if (sms <= 0) return MQA_ERR_CUDA;
-  int grid = sms * (use_tc ? tc_ctas_per_sm(hq) : simt_ctas_per_sm(dtype, d_k, hq));
+  int grid = sms * (use_tc ? tc_ctas_per_sm(hq) : simt_ctas_per_sm(dtype, d_k, d_v, hq));
   if (grid > kMaxCtas) grid = kMaxCtas;
   while (grid > 1 && scratch_bytes(b, g, hq, d_v, segs + size_t(grid)) > size_t(MQA_NOALLOC_SCRATCH_BYTES)) {
     const int step = grid / 8 > 0 ? grid / 8 : 1;
@@ -116,7 +116,7 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.h = h;
   a.g = g;
   a.m_max = m_max;
-  a.d = d_k;
+  a.d = d_v;   // the tensor-core path has d_k == d_v
   a.hq = hq;
   a.window = 0;
   a.q_beams = 0;
@@ -130,7 +130,7 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.ws = carve(scratch, b, g, hq, segs + size_t(grid));
   a.flags = status_flags;
   a.grid = grid;
-  cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, dtype, stream);
+  cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, d_k, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;
   if (launch_merge(a, dtype, stream) != cudaSuccess) return MQA_ERR_CUDA;
   return MQA_OK;

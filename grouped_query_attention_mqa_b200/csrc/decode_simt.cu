@@ -13,7 +13,9 @@
 //
 // This path is meant for h/g * d small enough that the arithmetic per byte
 // stays under the FFMA roofline (MHA is 1 FLOP/byte in bf16); larger groups
-// in bf16 go to the tensor-core kernel.
+// in bf16 go to the tensor-core kernel.  Keys and values may have different
+// widths (d_k for q and K, d_v for V and o), as the paper's per-head
+// dimensions k and v allow (velog paper review §2.4 and §3).
 #include "common.cuh"
 
 namespace mqa {
@@ -31,42 +33,77 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-template <typename T, int D>
+// Shared memory: reduction scratch, q [hq][DK] fp32, logits [hq][kTile],
+// m/l/alpha [hq], then two K stages of kTile rows of DK and two V stages of
+// kTile rows of DV (K0 K1 V0 V1).
+template <typename T, int DK, int DV>
 struct SimtLayout {
-  static constexpr int kRowBytes = D * int(sizeof(T)) + 16;   // +16: rows land on rotating banks
-  static constexpr int kChunks = D * int(sizeof(T)) / 16;     // 16-byte pieces per row
+  static constexpr int kRowBytesK = DK * int(sizeof(T)) + 16;   // +16: rows land on rotating banks
+  static constexpr int kRowBytesV = DV * int(sizeof(T)) + 16;
+  static constexpr int kChunksK = DK * int(sizeof(T)) / 16;     // 16-byte pieces per row
+  static constexpr int kChunksV = DV * int(sizeof(T)) / 16;
+  static constexpr int kStageK = kTile * kRowBytesK;
+  static constexpr int kStageV = kTile * kRowBytesV;
   static constexpr int kRedBytes = ((kThreads / 32 + kThreads + 2) * 8 + 15) / 16 * 16;
   static __host__ __device__ size_t bytes(int hq) {
-    return size_t(kRedBytes) + size_t(hq) * D * 4 + size_t(hq) * kTile * 4 + (size_t(3 * hq) * 4 + 15) / 16 * 16 +
-           size_t(4) * kTile * kRowBytes;
+    return size_t(kRedBytes) + size_t(hq) * DK * 4 + size_t(hq) * kTile * 4 + (size_t(3 * hq) * 4 + 15) / 16 * 16 +
+           size_t(2) * (kStageK + kStageV);
   }
 };
+
+// Stage `rows` rows of one cache (D elements each, row r at element
+// (row_base + r*g) * D) at a pitch of kRowBytes; row `new_row`, if any, comes
+// from `src_new` and is also written into the cache.
+template <typename T, int D, int kRowBytes>
+__device__ __forceinline__ void stage_rows(unsigned char* st, const T* __restrict__ C, int64_t row_base, int g,
+                                           int rows, int new_row, const T* __restrict__ src_new) {
+  constexpr int kChunks = D * int(sizeof(T)) / 16;
+  const int n = rows * kChunks;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const int r = i / kChunks, c = i - r * kChunks;
+    const int64_t off = (row_base + int64_t(r) * g) * D;
+    if (r == new_row) {
+      const uint4 x = reinterpret_cast<const uint4*>(src_new)[c];
+      reinterpret_cast<uint4*>(const_cast<T*>(C) + off)[c] = x;
+      *reinterpret_cast<uint4*>(st + r * kRowBytes + c * 16) = x;
+    } else {
+      cp_async16(st + r * kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(C + off) + c * 16);
+    }
+  }
+}
 
 // Stage the valid rows of a tile.  With the fused append (knew != nullptr)
 // the sequence's last tile holds its newest row: that row is taken from
 // knew/vnew, written into the cache and into the stage directly.
-template <typename T, int D>
+template <typename T, int DK, int DV>
 __device__ __forceinline__ void load_tile(unsigned char* ks, unsigned char* vs, const T* __restrict__ K,
                                           const T* __restrict__ V, const TileCoord& tc, int g, int m_max,
                                           const T* __restrict__ knew, const T* __restrict__ vnew) {
-  using L = SimtLayout<T, D>;
-  const int n = tc.rows * L::kChunks;
+  using L = SimtLayout<T, DK, DV>;
   const int64_t row_base = (int64_t(tc.seq) * m_max + tc.row0) * g + tc.head;
   const int new_row = (knew != nullptr && tc.k == tc.nb - 1) ? tc.rows - 1 : -1;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    const int r = i / L::kChunks, c = i - r * L::kChunks;
-    const int64_t off = (row_base + int64_t(r) * g) * D;        // element offset of the row
-    if (r == new_row) {
-      const int64_t src = (int64_t(tc.seq) * g + tc.head) * D;
-      const uint4 kv = reinterpret_cast<const uint4*>(knew + src)[c];
-      const uint4 vv = reinterpret_cast<const uint4*>(vnew + src)[c];
-      reinterpret_cast<uint4*>(const_cast<T*>(K) + off)[c] = kv;
-      reinterpret_cast<uint4*>(const_cast<T*>(V) + off)[c] = vv;
-      *reinterpret_cast<uint4*>(ks + r * L::kRowBytes + c * 16) = kv;
-      *reinterpret_cast<uint4*>(vs + r * L::kRowBytes + c * 16) = vv;
-    } else {
-      cp_async16(ks + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(K + off) + c * 16);
-      cp_async16(vs + r * L::kRowBytes + c * 16, reinterpret_cast<const unsigned char*>(V + off) + c * 16);
+  if constexpr (DK != DV) {
+    const int64_t src = int64_t(tc.seq) * g + tc.head;   // row of k_new / v_new
+    stage_rows<T, DK, L::kRowBytesK>(ks, K, row_base, g, tc.rows, new_row, knew ? knew + src * DK : nullptr);
+    stage_rows<T, DV, L::kRowBytesV>(vs, V, row_base, g, tc.rows, new_row, vnew ? vnew + src * DV : nullptr);
+  } else {
+    constexpr int D = DK;   // equal widths: one pass stages a K and a V piece per index
+    const int n = tc.rows * L::kChunksK;
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const int r = i / L::kChunksK, c = i - r * L::kChunksK;
+      const int64_t off = (row_base + int64_t(r) * g) * D;        // element offset of the row
+      if (r == new_row) {
+        const int64_t src = (int64_t(tc.seq) * g + tc.head) * D;
+        const uint4 kv = reinterpret_cast<const uint4*>(knew + src)[c];
+        const uint4 vv = reinterpret_cast<const uint4*>(vnew + src)[c];
+        reinterpret_cast<uint4*>(const_cast<T*>(K) + off)[c] = kv;
+        reinterpret_cast<uint4*>(const_cast<T*>(V) + off)[c] = vv;
+        *reinterpret_cast<uint4*>(ks + r * L::kRowBytesK + c * 16) = kv;
+        *reinterpret_cast<uint4*>(vs + r * L::kRowBytesV + c * 16) = vv;
+      } else {
+        cp_async16(ks + r * L::kRowBytesK + c * 16, reinterpret_cast<const unsigned char*>(K + off) + c * 16);
+        cp_async16(vs + r * L::kRowBytesV + c * 16, reinterpret_cast<const unsigned char*>(V + off) + c * 16);
+      }
     }
   }
 }
@@ -125,19 +162,20 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
 }
 __device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 
-template <typename T, int D>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs a) {
-  using L = SimtLayout<T, D>;
+  using L = SimtLayout<T, DK, DV>;
   extern __shared__ __align__(16) unsigned char smem[];
   int64_t* red = reinterpret_cast<int64_t*>(smem);
   float* q_s = reinterpret_cast<float*>(smem + L::kRedBytes);
-  float* p_s = q_s + a.hq * D;
+  float* p_s = q_s + a.hq * DK;
   float* m_s = p_s + a.hq * kTile;
   float* l_s = m_s + a.hq;
   float* al_s = l_s + a.hq;
   unsigned char* stage = reinterpret_cast<unsigned char*>(m_s) + (size_t(3 * a.hq) * 4 + 15) / 16 * 16;
-  // stage s: K at stage + s*kStageBytes, V at stage + (2+s)*kStageBytes
-  constexpr int kStageBytes = kTile * L::kRowBytes;
+  // stage s: K at stage + s*kStageK, V at stage + 2*kStageK + s*kStageV
+  unsigned char* const kst = stage;
+  unsigned char* const vst = stage + 2 * L::kStageK;
 
   const T* __restrict__ Q = static_cast<const T*>(a.q);
   const T* __restrict__ K = static_cast<const T*>(a.k);
@@ -154,8 +192,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   if (a.no_merge) {   // no merge follows: empty sequences get their zero rows here
     for (int s = blockIdx.x; s < a.b; s += gridDim.x) {
       if (clamp_len(__ldg(a.lens + s), a.m_max, nullptr, false) == 0) {
-        T* o = static_cast<T*>(a.o) + int64_t(s) * a.h * D;
-        for (int k = threadIdx.x; k < a.h * D; k += kThreads) o[k] = from_f32<T>(0.f);
+        T* o = static_cast<T*>(a.o) + int64_t(s) * a.h * DV;
+        for (int k = threadIdx.x; k < a.h * DV; k += kThreads) o[k] = from_f32<T>(0.f);
       }
     }
   }
@@ -169,11 +207,11 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   cursor_seek(cur, a.lens, g, a.m_max, a.window, kTile, sc.t_begin);
   {
     const TileCoord t0 = tile_coord(cur, g, kTile, sc.t_begin);
-    load_tile<T, D>(stage, stage + 2 * kStageBytes, K, V, t0, g, a.m_max, KN, VN);
+    load_tile<T, DK, DV>(kst, vst, K, V, t0, g, a.m_max, KN, VN);
     cp_async_commit();
   }
 
-  const int pairs_out = hq * (D / 2);
+  const int pairs_out = hq * (DV / 2);
   float2 acc[kMaxOutPairs];
 #pragma unroll
   for (int r = 0; r < kMaxOutPairs; ++r) acc[r] = make_float2(0.f, 0.f);
@@ -188,8 +226,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
     const TileCoord tc = tile_coord(cur, g, kTile, t);
 
     if (t == sc.t_begin || tc.k == 0) {   // a new segment starts: its queries, fresh state
-      const T* qg = Q + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq) * D;
-      for (int i = threadIdx.x; i < hq * D; i += kThreads) q_s[i] = to_f32(qg[i]) * qscale;
+      const T* qg = Q + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq) * DK;
+      for (int i = threadIdx.x; i < hq * DK; i += kThreads) q_s[i] = to_f32(qg[i]) * qscale;
       for (int i = threadIdx.x; i < hq; i += kThreads) {
         m_s[i] = -INFINITY;
         l_s[i] = 0.f;
@@ -200,8 +238,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
     if (t + 1 < sc.t_end) {
       cursor_seek(nxt, a.lens, g, a.m_max, a.window, kTile, t + 1);
       const TileCoord tn = tile_coord(nxt, g, kTile, t + 1);
-      load_tile<T, D>(stage + (st ^ 1) * kStageBytes, stage + (2 + (st ^ 1)) * kStageBytes, K, V, tn, g,
-                      a.m_max, KN, VN);
+      load_tile<T, DK, DV>(kst + (st ^ 1) * L::kStageK, vst + (st ^ 1) * L::kStageV, K, V, tn, g, a.m_max, KN,
+                           VN);
     }
     cp_async_commit();
     cp_async_wait1();
@@ -212,7 +250,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
       const int i = p / kTile, r = p - i * kTile;
       const int part = threadIdx.x % split;
       float s = 0.f;
-      if (r < tc.rows) s = dot_row<T>(q_s + i * D, stage + st * kStageBytes + r * L::kRowBytes, part * (D / split), D / split);
+      if (r < tc.rows)
+        s = dot_row<T>(q_s + i * DK, kst + st * L::kStageK + r * L::kRowBytesK, part * (DK / split), DK / split);
       for (int o = split / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (part == 0) p_s[i * kTile + r] = r < tc.rows ? s : -INFINITY;
     }
@@ -246,14 +285,14 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
     for (int r = 0; r < kMaxOutPairs; ++r) {
       const int f = threadIdx.x + r * kThreads;
       if (f < pairs_out) {
-        const int i = f / (D / 2), c2 = f - i * (D / 2);
+        const int i = f / (DV / 2), c2 = f - i * (DV / 2);
         const float alpha = al_s[i];
         float2 o2 = make_float2(acc[r].x * alpha, acc[r].y * alpha);
         const float* pw = p_s + i * kTile;
-        const unsigned char* vrow = stage + (2 + st) * kStageBytes;
+        const unsigned char* vrow = vst + st * L::kStageV;
         for (int row = 0; row < tc.rows; ++row) {
           const float w = pw[row];
-          const float2 v = load_v_pair(vrow + row * L::kRowBytes, c2, static_cast<T*>(nullptr));
+          const float2 v = load_v_pair(vrow + row * L::kRowBytesV, c2, static_cast<T*>(nullptr));
           o2.x = fmaf(w, v.x, o2.x);
           o2.y = fmaf(w, v.y, o2.y);
         }
@@ -270,13 +309,13 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
       for (int r = 0; r < kMaxOutPairs; ++r) {
         const int f = threadIdx.x + r * kThreads;
         if (f < pairs_out) {
-          const int i = f / (D / 2), c2 = f - i * (D / 2);
+          const int i = f / (DV / 2), c2 = f - i * (DV / 2);
           const float inv = 1.f / l_s[i];
           const float2 v = make_float2(acc[r].x * inv, acc[r].y * inv);
           if (whole) {
-            store_pair(O + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq + i) * D + 2 * c2, v);
+            store_pair(O + (int64_t(tc.seq) * a.h + int64_t(tc.head) * hq + i) * DV + 2 * c2, v);
           } else {
-            *reinterpret_cast<float2*>(a.ws.part_o + (slot * hq + i) * D + 2 * c2) = v;
+            *reinterpret_cast<float2*>(a.ws.part_o + (slot * hq + i) * DV + 2 * c2) = v;
           }
         }
       }
@@ -292,7 +331,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
 }
 
 // Opt the kernel into large dynamic shared memory once per device.
-template <typename T, int D>
+template <typename T, int DK, int DV>
 cudaError_t ensure_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
@@ -302,15 +341,15 @@ cudaError_t ensure_smem_attr() {
   int optin = 0;
   e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_simt_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  e = cudaFuncSetAttribute(decode_simt_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }
 
-template <typename T, int D>
+template <typename T, int DK, int DV>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
-  const size_t smem = SimtLayout<T, D>::bytes(a.hq);
-  cudaError_t e = ensure_smem_attr<T, D>();
+  const size_t smem = SimtLayout<T, DK, DV>::bytes(a.hq);
+  cudaError_t e = ensure_smem_attr<T, DK, DV>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(a.grid));
@@ -322,63 +361,77 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_simt_kernel<T, D>, a);
+  return cudaLaunchKernelEx(&cfg, decode_simt_kernel<T, DK, DV>, a);
 }
 
 // Resident CTAs per SM for this shared-memory size, cached per (device, h/g).
-template <typename T, int D>
+template <typename T, int DK, int DV>
 int occupancy_t(int hq) {
   static int cache[64][129] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   const bool cacheable = dev >= 0 && dev < 64 && hq >= 1 && hq <= 128;
   if (cacheable && cache[dev][hq] > 0) return cache[dev][hq];
-  const size_t smem = SimtLayout<T, D>::bytes(hq);
-  if (ensure_smem_attr<T, D>() != cudaSuccess) return 1;
+  const size_t smem = SimtLayout<T, DK, DV>::bytes(hq);
+  if (ensure_smem_attr<T, DK, DV>() != cudaSuccess) return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_simt_kernel<T, D>, kThreads, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_simt_kernel<T, DK, DV>, kThreads, smem) !=
+          cudaSuccess ||
       n < 1)
     n = 1;
   if (cacheable) cache[dev][hq] = n;
   return n;
 }
 
-}  // namespace
-
-cudaError_t launch_decode_simt(const DecodeArgs& a, mqa_dtype_t dtype, cudaStream_t stream) {
-  if (dtype == MQA_BF16) {
-    switch (a.d) {
-      case 32: return launch_t<__nv_bfloat16, 32>(a, stream);
-      case 64: return launch_t<__nv_bfloat16, 64>(a, stream);
-      case 128: return launch_t<__nv_bfloat16, 128>(a, stream);
-    }
-  } else {
-    switch (a.d) {
-      case 32: return launch_t<float, 32>(a, stream);
-      case 64: return launch_t<float, 64>(a, stream);
-      case 128: return launch_t<float, 128>(a, stream);
-    }
+// The built widths: d_k, d_v in {32, 64, 128}, any pairing.
+template <typename T, int DK>
+cudaError_t launch_dk(const DecodeArgs& a, int d_v, cudaStream_t stream) {
+  switch (d_v) {
+    case 32: return launch_t<T, DK, 32>(a, stream);
+    case 64: return launch_t<T, DK, 64>(a, stream);
+    case 128: return launch_t<T, DK, 128>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+template <typename T>
+cudaError_t launch_typed(const DecodeArgs& a, int d_k, int d_v, cudaStream_t stream) {
+  switch (d_k) {
+    case 32: return launch_dk<T, 32>(a, d_v, stream);
+    case 64: return launch_dk<T, 64>(a, d_v, stream);
+    case 128: return launch_dk<T, 128>(a, d_v, stream);
   }
   return cudaErrorInvalidValue;
 }
 
-int simt_tile_rows() { return kTile; }
-
-int simt_ctas_per_sm(mqa_dtype_t dtype, int d, int hq) {
-  if (dtype == MQA_BF16) {
-    switch (d) {
-      case 32: return occupancy_t<__nv_bfloat16, 32>(hq);
-      case 64: return occupancy_t<__nv_bfloat16, 64>(hq);
-      case 128: return occupancy_t<__nv_bfloat16, 128>(hq);
-    }
-  } else {
-    switch (d) {
-      case 32: return occupancy_t<float, 32>(hq);
-      case 64: return occupancy_t<float, 64>(hq);
-      case 128: return occupancy_t<float, 128>(hq);
-    }
+template <typename T, int DK>
+int occupancy_dk(int d_v, int hq) {
+  switch (d_v) {
+    case 32: return occupancy_t<T, DK, 32>(hq);
+    case 64: return occupancy_t<T, DK, 64>(hq);
+    case 128: return occupancy_t<T, DK, 128>(hq);
   }
   return 1;
+}
+template <typename T>
+int occupancy_typed(int d_k, int d_v, int hq) {
+  switch (d_k) {
+    case 32: return occupancy_dk<T, 32>(d_v, hq);
+    case 64: return occupancy_dk<T, 64>(d_v, hq);
+    case 128: return occupancy_dk<T, 128>(d_v, hq);
+  }
+  return 1;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, int d_k, mqa_dtype_t dtype, cudaStream_t stream) {
+  return dtype == MQA_BF16 ? launch_typed<__nv_bfloat16>(a, d_k, a.d, stream) : launch_typed<float>(a, d_k, a.d, stream);
+}
+
+int simt_tile_rows() { return kTile; }
+
+int simt_ctas_per_sm(mqa_dtype_t dtype, int d_k, int d_v, int hq) {
+  return dtype == MQA_BF16 ? occupancy_typed<__nv_bfloat16>(d_k, d_v, hq) : occupancy_typed<float>(d_k, d_v, hq);
 }
 
 }  // namespace mqa

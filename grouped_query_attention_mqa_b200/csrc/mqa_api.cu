@@ -88,10 +88,10 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
     return MQA_ERR_INVALID_ARG;
   const int hq = h / g;
   if (workspace_bytes_given < workspace_bytes(b, g, hq, d_v)) return MQA_ERR_INVALID_ARG;
-  if (d_k != d_v || (d_k != 32 && d_k != 64 && d_k != 128)) return MQA_ERR_UNSUPPORTED;
+  if ((d_k != 32 && d_k != 64 && d_k != 128) || (d_v != 32 && d_v != 64 && d_v != 128)) return MQA_ERR_UNSUPPORTED;
 
-  const bool tc_ok = dtype == MQA_BF16 && tc_supported(d_k, hq);
-  const bool simt_ok = int64_t(hq) * d_k <= 4096;
+  const bool tc_ok = dtype == MQA_BF16 && d_k == d_v && tc_supported(d_k, hq);
+  const bool simt_ok = int64_t(hq) * d_k <= 4096 && int64_t(hq) * d_v <= 4096;
   bool use_tc;
   if (path == MQA_PATH_TCGEN05) {
     if (!tc_ok) return MQA_ERR_UNSUPPORTED;
@@ -118,7 +118,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.h = h;
   a.g = g;
   a.m_max = m_max;
-  a.d = d_k;
+  a.d = d_v;   // the tensor-core path has d_k == d_v
   a.hq = hq;
   a.window = opts ? opts->window : 0;
   a.q_beams = 0;
@@ -135,10 +135,10 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.ws = carve_workspace(workspace, b, g, hq);
   a.flags = status_flags;
   int grid = opts && opts->num_ctas > 0 ? opts->num_ctas
-                                         : sms * (use_tc ? tc_ctas_per_sm(hq) : simt_ctas_per_sm(dtype, d_k, hq));
+                                         : sms * (use_tc ? tc_ctas_per_sm(hq) : simt_ctas_per_sm(dtype, d_k, d_v, hq));
   a.grid = grid < 1 ? 1 : (grid > kMaxCtas ? kMaxCtas : grid);
 
-  cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, dtype, stream);
+  cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, d_k, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;
   if (!a.no_merge) e = launch_merge(a, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;

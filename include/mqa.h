@@ -149,8 +149,11 @@ MQA_API size_t mqa_decode_workspace_size(int b, int h, int g, int d_v);
  *                    aligned; contents on entry do not matter; calls that
  *                    share a workspace must be ordered on one stream
  *   status_flags     device int32 or NULL (see above)
- * Supported: h % g == 0, d_k == d_v in {32, 64, 128}; the SIMT path takes
- * h/g * d_v <= 4096, the tensor-core path bf16 with d = 128 and h/g <= 64.  b = 0 is a no-op returning MQA_OK.
+ * Supported: h % g == 0, d_k and d_v in {32, 64, 128}, in any pairing (the
+ * paper's per-head key size k and value size v are independent).  The SIMT
+ * path takes h/g * d_k <= 4096 and h/g * d_v <= 4096; the tensor-core path
+ * bf16 with d_k = d_v = 128 and h/g <= 64 (with d_k != d_v the automatic
+ * choice is the SIMT path).  b = 0 is a no-op returning MQA_OK.
  * Errors: MQA_ERR_INVALID_ARG (NULL pointer, h % g != 0, non-finite scale,
  * workspace too small or misaligned), MQA_ERR_UNSUPPORTED (head sizes or
  * group widths not built), MQA_ERR_CUDA (launch failure).
@@ -179,8 +182,9 @@ MQA_API mqa_status_t mqa_decode_ex(void* o, const void* q, const void* k_cache, 
  * the CTA that loads a sequence's last tile first writes the new row into the
  * cache, then attends over it.
  *
- *   k_cache, v_cache  device [b, m_max, g, d]   read, and row lens[b]-1 written
- *   k_new, v_new      device [b, g, d]          read
+ *   k_cache, v_cache  device [b, m_max, g, d_k], [b, m_max, g, d_v]
+ *                     read, and row lens[b]-1 written
+ *   k_new, v_new      device [b, g, d_k], [b, g, d_v]   read
  *   other arguments as for mqa_decode_ex; lens outside [1, m_max] are clamped
  *   and flagged as there (the row then goes to the clamped length minus one;
  *   a sequence whose clamped length is 0 writes nothing and outputs zeros).

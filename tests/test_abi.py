@@ -84,7 +84,11 @@ def test_decode_rejects_bad_arguments_without_launching(lib):
     assert _decode(lib, dtype=7) == INV
     assert _decode(lib, m_max=0) == INV
     assert _decode(lib, d_k=96, d_v=96) == UNS           # head size not built
-    assert _decode(lib, d_k=128, d_v=64) == UNS          # d_k != d_v not built
+    assert _decode(lib, d_k=128, d_v=96) == UNS          # value width not built
+    opts = binding.DecodeOptions(2, 0)                   # tensor cores: d_k = d_v only
+    assert _decode(lib, d_k=128, d_v=64, opts=ctypes.byref(opts)) == UNS
+    opts = binding.DecodeOptions(1, 0)                   # SIMT: h/g * d_v <= 4096 as well
+    assert _decode(lib, h=64, d_k=32, d_v=128, opts=ctypes.byref(opts)) == UNS
     opts = binding.DecodeOptions(9, 0)
     assert _decode(lib, opts=ctypes.byref(opts)) == INV  # unknown path
     opts = binding.DecodeOptions(0, binding.MQA_MAX_CTAS + 1)
