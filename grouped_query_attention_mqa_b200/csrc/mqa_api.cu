@@ -100,7 +100,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
     if (!simt_ok) return MQA_ERR_UNSUPPORTED;
     use_tc = false;
   } else {
-    use_tc = tc_ok && hq >= 8;
+    use_tc = tc_ok;
     if (!use_tc && !simt_ok) return MQA_ERR_UNSUPPORTED;
   }
 

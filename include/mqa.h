@@ -72,7 +72,7 @@ typedef enum {
 
 /* Kernel path of mqa_decode_ex. */
 typedef enum {
-  MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d = 128 and h/g >= 8  */
+  MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d = 128, h/g <= 64     */
   MQA_PATH_SIMT = 1,         /* CUDA-core FFMA path (any dtype, h/g*d <= 4096) */
   MQA_PATH_TCGEN05 = 2       /* tcgen05 tensor-core path (bf16, d = 128,
                                 h/g <= 64)                                    */

@@ -96,6 +96,21 @@ def test_decode_matches_oracle(shape, num_ctas):
     assert_close(out, ref, wl.dtype, wl.name)
 
 
+@pytest.mark.parametrize("hq", [1, 2, 4])
+def test_automatic_path_takes_tensor_cores_for_small_groups(hq):
+    """bf16, d = 128: the automatic choice is the tensor-core kernel at every
+    group width it serves, MHA (h/g = 1) included, where it streams the cache
+    at more than twice the CUDA-core kernel's rate.  Same path and CTA count
+    give the same bits."""
+    wl = small("bf16", 4, 8, 8 // hq, 128, 400, 1, 400)
+    if not tc_available(wl):
+        pytest.skip("tensor-core path not built")
+    auto, ref = run_case(wl, seed=hq, path="auto")
+    tc, _ = run_case(wl, seed=hq, path="tcgen05")
+    assert np.array_equal(auto, tc)
+    assert_close(auto, ref, "bf16", f"auto hq={hq}")
+
+
 @pytest.mark.parametrize("path", ["simt", "tcgen05"])
 @pytest.mark.parametrize("hq", [1, 4, 8, 12, 16, 32, 48, 64])
 def test_both_paths_on_group_widths(path, hq):
