@@ -11,11 +11,11 @@
 // all heads of the group), and an online softmax keeps a running max m and sum
 // l per head.  Exponentials are exp2 of log2(e)-prescaled logits.
 //
-// This path is meant for h/g * d small enough that the arithmetic per byte
-// stays under the FFMA roofline (MHA is 1 FLOP/byte in bf16); larger groups
-// in bf16 go to the tensor-core kernel.  Keys and values may have different
-// widths (d_k for q and K, d_v for V and o), as the paper's per-head
-// dimensions k and v allow (velog paper review §2.4 and §3).
+// The arithmetic is h/g FLOP per cache byte in bf16, so this kernel keeps up
+// with HBM only for small groups; bf16 with d = 128 is served by the
+// tensor-core kernel, and this one takes fp32, head sizes 32 and 64, and keys
+// and values of different widths (d_k for q and K, d_v for V and o), as the
+// paper's per-head dimensions k and v allow (velog paper review §2.4, §3).
 #include "common.cuh"
 
 namespace mqa {
