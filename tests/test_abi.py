@@ -102,6 +102,31 @@ def test_decode_rejects_bad_arguments_without_launching(lib):
     assert _decode(lib, b=0) == binding.MQA_OK           # empty batch: nothing to do
 
 
+def _noalloc(lib, **kw):
+    a = dict(o=FAKE, q=FAKE, k=FAKE, v=FAKE, lens=FAKE, b=2, h=8, g=1, m_max=16, d_k=128, d_v=128, scale=1.0,
+             dtype=binding.MQA_BF16, flags=None, stream=None)
+    a.update(kw)
+    return lib.mqa_decode_noalloc(a["o"], a["q"], a["k"], a["v"], a["lens"], a["b"], a["h"], a["g"], a["m_max"],
+                                  a["d_k"], a["d_v"], a["scale"], a["dtype"], a["flags"], a["stream"])
+
+
+def test_noalloc_rejects_bad_arguments_without_launching(lib):
+    """mqa_decode_noalloc checks its arguments as mqa_decode does, before it
+    touches the device; every call below fails a check."""
+    INV, UNS = binding.MQA_ERR_INVALID_ARG, binding.MQA_ERR_UNSUPPORTED
+    assert _noalloc(lib, g=3) == INV                     # h % g != 0
+    assert _noalloc(lib, lens=None) == INV
+    assert _noalloc(lib, q=ctypes.c_void_p(0x10008)) == INV        # misaligned
+    assert _noalloc(lib, scale=float("nan")) == INV
+    assert _noalloc(lib, dtype=7) == INV
+    assert _noalloc(lib, m_max=0) == INV
+    assert _noalloc(lib, d_k=96, d_v=96) == UNS          # head size not built
+    assert _noalloc(lib, d_k=128, d_v=48) == UNS         # value width not built
+    assert _noalloc(lib, h=64, d_k=32, d_v=128) == UNS   # SIMT (unequal widths): h/g * d_v > 4096
+    assert _noalloc(lib, b=4096, h=64, g=64) == INV      # partials beyond the 16 MiB array
+    assert _noalloc(lib, b=0) == binding.MQA_OK          # empty batch: nothing to do
+
+
 def test_append_rejects_bad_arguments_without_launching(lib):
     INV = binding.MQA_ERR_INVALID_ARG
     f = lib.mqa_kv_append
