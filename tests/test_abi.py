@@ -127,6 +127,55 @@ def test_noalloc_rejects_bad_arguments_without_launching(lib):
     assert _noalloc(lib, b=0) == binding.MQA_OK          # empty batch: nothing to do
 
 
+def _fused(lib, **kw):
+    a = dict(o=FAKE, q=FAKE, k=FAKE, v=FAKE, kn=FAKE, vn=FAKE, lens=FAKE, b=2, h=8, g=1, m_max=16, d_k=128, d_v=128,
+             scale=1.0, dtype=binding.MQA_BF16, ws=FAKE, ws_bytes=1 << 40, flags=None, opts=None, stream=None)
+    a.update(kw)
+    return lib.mqa_decode_append(a["o"], a["q"], a["k"], a["v"], a["kn"], a["vn"], a["lens"], a["b"], a["h"], a["g"],
+                                 a["m_max"], a["d_k"], a["d_v"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"],
+                                 a["flags"], a["opts"], a["stream"])
+
+
+def test_fused_step_rejects_bad_arguments_without_launching(lib):
+    INV, UNS = binding.MQA_ERR_INVALID_ARG, binding.MQA_ERR_UNSUPPORTED
+    assert _fused(lib, kn=None) == INV                   # the new rows are required
+    assert _fused(lib, vn=None) == INV
+    assert _fused(lib, kn=ctypes.c_void_p(0x10004)) == INV         # misaligned new row
+    assert _fused(lib, g=3) == INV
+    assert _fused(lib, ws_bytes=100) == INV
+    assert _fused(lib, d_k=96, d_v=96) == UNS
+    opts = binding.DecodeOptions(2, 0)                   # tensor cores: d_k = d_v only
+    assert _fused(lib, d_v=64, opts=ctypes.byref(opts)) == UNS
+    assert _fused(lib, b=0, kn=None, vn=None) == binding.MQA_OK
+
+
+def _beam(lib, **kw):
+    a = dict(o=FAKE, q=FAKE, pk=FAKE, pv=FAKE, pl=FAKE, sk=FAKE, sv=FAKE, sl=FAKE, b=2, W=4, h=8, g=1, m_p=64, m_s=8,
+             d_k=128, d_v=128, scale=1.0, dtype=binding.MQA_BF16, ws=FAKE, ws_bytes=1 << 40, flags=None, stream=None)
+    a.update(kw)
+    return lib.mqa_decode_beam(a["o"], a["q"], a["pk"], a["pv"], a["pl"], a["sk"], a["sv"], a["sl"], a["b"], a["W"],
+                               a["h"], a["g"], a["m_p"], a["m_s"], a["d_k"], a["d_v"], a["scale"], a["dtype"], a["ws"],
+                               a["ws_bytes"], a["flags"], a["stream"])
+
+
+def test_beam_rejects_bad_arguments_without_launching(lib):
+    INV, UNS = binding.MQA_ERR_INVALID_ARG, binding.MQA_ERR_UNSUPPORTED
+    ws = lib.mqa_decode_beam_workspace_size
+    assert ws(2, 4, 8, 1, 128) == lib.mqa_decode_workspace_size(2, 32, 1, 128)   # W beams' heads share a segment
+    assert ws(2, 0, 8, 1, 128) == 0 and ws(2, 4, 8, 3, 128) == 0
+    assert _beam(lib, W=0) == INV
+    assert _beam(lib, m_s=0) == INV
+    assert _beam(lib, sl=None) == INV
+    assert _beam(lib, sk=ctypes.c_void_p(0x10008)) == INV          # misaligned suffix cache
+    assert _beam(lib, ws=ctypes.c_void_p(0x10010)) == INV          # workspace not 256-aligned
+    assert _beam(lib, ws_bytes=ws(2, 4, 8, 1, 128) - 1) == INV     # one byte short
+    assert _beam(lib, scale=float("inf")) == INV
+    assert _beam(lib, dtype=binding.MQA_F32) == UNS      # tensor cores only: bf16
+    assert _beam(lib, d_k=64, d_v=64) == UNS             # d = 128 only
+    assert _beam(lib, W=16, h=8) == UNS                  # W * h/g = 128 > 64 query columns
+    assert _beam(lib, b=0) == binding.MQA_OK
+
+
 def test_append_rejects_bad_arguments_without_launching(lib):
     INV = binding.MQA_ERR_INVALID_ARG
     f = lib.mqa_kv_append
