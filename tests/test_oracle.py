@@ -174,6 +174,29 @@ def test_weights_sum_to_one_and_match_lse(hq, g, L, seed):
         np.testing.assert_allclose(np.exp(s - lse[0, i]), w[0][i], rtol=1e-12, atol=1e-15)
 
 
+@settings(max_examples=25, deadline=None)
+@given(hq=st.sampled_from([1, 3]), g=st.sampled_from([1, 2]), dk=st.sampled_from([2, 5]),
+       dv=st.sampled_from([1, 3, 6]), L=st.integers(1, 10), seed=st.integers(0, 10**6))
+def test_output_is_a_convex_combination_of_the_valid_v_rows(hq, g, dk, dv, L, seed):
+    """Each output is a weighted mean of its group's valid V rows, so every
+    column lies between that column's minimum and maximum over those rows,
+    whatever d_k and d_v are; rows past the length hold values far outside the
+    range and must not pull the output out of it."""
+    rng = np.random.default_rng(seed)
+    h, m = hq * g, 12
+    q = _rand(rng, 2, h, dk) * 3.0
+    K = _rand(rng, 2, m, g, dk)
+    V = _rand(rng, 2, m, g, dv)
+    V[:, L:] = 1e6
+    o, _ = oracle_decode(q, K, V, [L, L], g=g, scale=0.9)
+    assert o.shape == (2, h, dv)
+    for bi in range(2):
+        for i in range(h):
+            rows = V[bi, :L, i // hq]
+            assert np.all(o[bi, i] >= rows.min(axis=0) - 1e-12)
+            assert np.all(o[bi, i] <= rows.max(axis=0) + 1e-12)
+
+
 def test_length_one_cache_returns_v():
     """A softmax over one row is 1, so each head's output is that row of V."""
     rng = np.random.default_rng(4)
