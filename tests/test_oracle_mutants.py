@@ -1,10 +1,13 @@
-"""The oracle's pins catch plausible mistakes.  Each mutant below is a decode
-written here with one slip planted (on the CPU, never in the oracle itself):
-a wrong query-head -> K/V-head map, a dropped scale, no max-subtraction, rows
-past the length attended, K weighted instead of V, and a step that attends
-before it appends.  The pins of test_oracle.py are run against each mutant and
-at least one must fail.  The same decode with no slip passes every pin, so a
-failure comes from the slip and not from the harness."""
+"""The oracle's pins catch plausible mistakes.  Each mutant below is a decode,
+prefill or beam step written here with one slip planted (on the CPU, never in
+the oracle itself): a wrong query-head -> K/V-head map, a dropped scale, no
+max-subtraction, rows past the length attended, K weighted instead of V, a local
+window one row too wide, a step that attends before it appends, a causal mask
+one row off, keys taken across
+sequence boundaries, another beam's suffix, a dropped prefix.  The pins of
+test_oracle.py are run against each mutant and at least one must fail.  The
+same code with no slip passes every pin, so a failure comes from the slip and
+not from the harness."""
 import numpy as np
 import pytest
 
@@ -12,15 +15,13 @@ import test_oracle as T
 from conftest import read_golden
 from oracle import oracle_decode, oracle_kv_append
 
-SLIPS = ["group", "no_scale", "no_max", "unmasked", "v_is_k"]
+SLIPS = ["group", "no_scale", "no_max", "unmasked", "v_is_k", "window_off_by_one"]
 
 
 def mutant_decode(slip):
     """Scaled masked softmax attention per (sequence, head), with `slip`
     planted (None: no slip)."""
     def decode(q, k_cache, v_cache, lens, g, scale, return_weights=False, window=0):
-        if window:
-            raise NotImplementedError("the pins run here use no window")
         q = np.asarray(q, np.float64)
         K = np.asarray(k_cache, np.float64)
         V = np.asarray(v_cache, np.float64)
@@ -34,17 +35,20 @@ def mutant_decode(slip):
                 L = int(lens[bi])
                 wb = np.zeros((h, max(L, 0)))
                 if L > 0:
-                    n = m if slip == "unmasked" else L
+                    lo = max(0, L - window) if window > 0 else 0
+                    if slip == "window_off_by_one" and window > 0:
+                        lo = max(0, lo - 1)
+                    hi = m if slip == "unmasked" else L
                     for i in range(h):
                         j = i % g if slip == "group" else i // hq
-                        Kj, Vj = K[bi, :n, j], V[bi, :n, j]
+                        Kj, Vj = K[bi, lo:hi, j], V[bi, lo:hi, j]
                         s = (Kj @ q[bi, i]) * (1.0 if slip == "no_scale" else scale)
                         mu = 0.0 if slip == "no_max" else s.max()
                         e = np.exp(s - mu)
                         w = e / e.sum()
                         o[bi, i] = w @ (Kj if slip == "v_is_k" else Vj)
                         lse[bi, i] = mu + np.log(e.sum())
-                        wb[i] = w[:L]
+                        wb[i, lo:L] = w[:L - lo]
                 weights.append(wb)
         return (o, lse, weights) if return_weights else (o, lse)
     return decode
@@ -78,12 +82,18 @@ PINS = [
     ("row permutation, V linearity", T.test_row_permutation_and_v_linearity),
     ("zero length", T.test_zero_length_gives_zero_row),
     ("append before attend", T.test_step_appends_before_attending),
+    ("window 1 returns the newest V row", lambda: T.test_window_one_returns_the_newest_row_of_v(read_golden)),
+    ("window covering the cache", lambda: T.test_window_covering_the_cache_is_full_attention(read_golden)),
+] + [
+    (f"window {w} brute force", lambda w=w: T.test_window_is_brute_force_on_the_newest_rows(w)) for w in (1, 3, 5, 32)
+] + [
+    ("window 32 = current + 31", T.test_notes_window_is_current_plus_31_previous),
 ]
 
 
-def failing_pins():
+def failing_pins(pins=None):
     failed = []
-    for name, pin in PINS:
+    for name, pin in PINS if pins is None else pins:
         try:
             pin()
         except Exception:   # an assertion, or the slip's own breakage (NaN, shape)
@@ -105,3 +115,97 @@ def test_a_pin_catches_the_planted_slip(monkeypatch, slip):
 def test_a_pin_catches_attending_before_appending(monkeypatch):
     monkeypatch.setattr(T, "oracle_decode_step", step_attend_then_append)
     assert failing_pins() == ["append before attend"]
+
+
+# ------------------------------------------------------------ prefill
+
+def mutant_prefill(slip):
+    """Per position t of each packed sequence: softmax attention over keys
+    0..t of that sequence (all n keys without the mask), with `slip` planted."""
+    def prefill(q, k, v, cu_seqlens, g, scale, causal=True):
+        q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+        cu = [int(x) for x in cu_seqlens]
+        T_, h, _ = q.shape
+        hq = h // g
+        o = np.zeros((T_, h, v.shape[2]))
+        lse = np.full((T_, h), -np.inf)
+        for si in range(len(cu) - 1):
+            a, n = cu[si], cu[si + 1] - cu[si]
+            for t in range(n):
+                last = t if causal else n - 1
+                if slip == "mask_off_by_one":
+                    last = min(last + 1, n - 1)
+                first = 0 if slip == "across_sequences" else a
+                for i in range(h):
+                    j = i % g if slip == "group" else i // hq
+                    s = (k[first:a + last + 1, j] @ q[a + t, i]) * scale
+                    mu = s.max()
+                    e = np.exp(s - mu)
+                    o[a + t, i] = (e / e.sum()) @ v[first:a + last + 1, j]
+                    lse[a + t, i] = mu + np.log(e.sum())
+        return o, lse
+    return prefill
+
+
+PREFILL_PINS = [
+    (f"prefill brute force h={h} g={g}", lambda h=h, g=g: T.test_prefill_is_brute_force_over_the_causal_prefix(h, g))
+    for h, g in [(4, 1), (4, 2), (4, 4)]
+] + [
+    ("prefill first position", T.test_prefill_first_position_returns_its_own_v),
+    ("prefill without mask", T.test_prefill_without_mask_sees_the_whole_sequence),
+    ("prefill causality", T.test_prefill_prefix_is_unchanged_by_later_tokens),
+    ("prefill last position == decode", T.test_prefill_last_position_is_the_decode_step),
+    ("prefill MQA == MHA", T.test_prefill_mqa_equals_mha_with_replicated_kv),
+]
+
+
+def test_prefill_mutant_without_a_slip_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(T, "oracle_prefill", mutant_prefill(None))
+    assert failing_pins(PREFILL_PINS) == []
+
+
+@pytest.mark.parametrize("slip", ["mask_off_by_one", "across_sequences", "group"])
+def test_a_prefill_pin_catches_the_planted_slip(monkeypatch, slip):
+    monkeypatch.setattr(T, "oracle_prefill", mutant_prefill(slip))
+    assert failing_pins(PREFILL_PINS), f"no prefill pin fails with the slip '{slip}'"
+
+
+# ------------------------------------------------------------ beams sharing a prefix
+
+def mutant_beam(slip):
+    """Beam (s, w) attends over sequence s's prefix rows, then the beam's own
+    suffix rows, with `slip` planted."""
+    def beam(q, prefix_k, prefix_v, prefix_lens, suffix_k, suffix_v, suffix_lens, g, scale):
+        q = np.asarray(q, np.float64)
+        b, W, h, _ = q.shape
+        o = np.zeros((b, W, h, np.asarray(prefix_v).shape[3]))
+        lse = np.full((b, W, h), -np.inf)
+        for si in range(b):
+            for w in range(W):
+                r = si * W + ((w + 1) % W if slip == "other_beam" else w)
+                lp = 0 if slip == "no_prefix" else int(prefix_lens[si])
+                K = np.concatenate([prefix_k[si, :lp], suffix_k[r, :int(suffix_lens[r])]])[None]
+                V = np.concatenate([prefix_v[si, :lp], suffix_v[r, :int(suffix_lens[r])]])[None]
+                if K.shape[1]:
+                    ob, lb = oracle_decode(q[si, w][None], K, V, [K.shape[1]], g, scale)
+                    o[si, w], lse[si, w] = ob[0], lb[0]
+        return o, lse
+    return beam
+
+
+BEAM_PINS = [
+    ("beam brute force", T.test_beam_is_brute_force_over_prefix_then_suffix),
+    ("beams with the same suffix agree", T.test_beams_with_the_same_suffix_agree),
+    ("beam with empty suffix or prefix", T.test_beam_with_empty_suffix_or_prefix_is_plain_decode),
+]
+
+
+def test_beam_mutant_without_a_slip_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(T, "oracle_decode_beam", mutant_beam(None))
+    assert failing_pins(BEAM_PINS) == []
+
+
+@pytest.mark.parametrize("slip", ["other_beam", "no_prefix"])
+def test_a_beam_pin_catches_the_planted_slip(monkeypatch, slip):
+    monkeypatch.setattr(T, "oracle_decode_beam", mutant_beam(slip))
+    assert failing_pins(BEAM_PINS), f"no beam pin fails with the slip '{slip}'"
