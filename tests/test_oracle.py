@@ -308,6 +308,7 @@ def test_append_is_the_concat_of_the_review():
     kn = rng.integers(0, 2**16, size=(b, g, d), dtype=np.uint16)
     vn = rng.integers(0, 2**16, size=(b, g, d), dtype=np.uint16)
     pos = np.array([0, 3, 5])
+    Kc0, Vc0 = Kc.copy(), Vc.copy()
     K2, V2 = oracle_kv_append(Kc, Vc, kn, vn, pos)
     for bi in range(b):
         L = pos[bi]
@@ -315,7 +316,7 @@ def test_append_is_the_concat_of_the_review():
         cat_v = np.concatenate([Vc[bi, :L], vn[bi][None]], axis=0)
         assert np.array_equal(K2[bi, :L + 1], cat_k) and np.array_equal(V2[bi, :L + 1], cat_v)
         assert np.array_equal(K2[bi, L + 1:], Kc[bi, L + 1:]) and np.array_equal(V2[bi, L + 1:], Vc[bi, L + 1:])
-    assert np.array_equal(Kc, Kc)  # inputs untouched (copy semantics)
+    assert np.array_equal(Kc, Kc0) and np.array_equal(Vc, Vc0)   # inputs untouched (copy semantics)
 
 
 def test_append_out_of_range_row_writes_nothing():

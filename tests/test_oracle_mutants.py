@@ -2,8 +2,8 @@
 prefill or beam step written here with one slip planted (on the CPU, never in
 the oracle itself): a wrong query-head -> K/V-head map, a dropped scale, no
 max-subtraction, rows past the length attended, K weighted instead of V, a local
-window one row too wide, a step that attends before it appends, a causal mask
-one row off, keys taken across
+window one row too wide, a step that attends before it appends, an append
+one row off, in place or without its range check, a causal mask one row off, keys taken across
 sequence boundaries, another beam's suffix, a dropped prefix.  The pins of
 test_oracle.py are run against each mutant and at least one must fail.  The
 same code with no slip passes every pin, so a failure comes from the slip and
@@ -209,3 +209,37 @@ def test_beam_mutant_without_a_slip_passes_every_pin(monkeypatch):
 def test_a_beam_pin_catches_the_planted_slip(monkeypatch, slip):
     monkeypatch.setattr(T, "oracle_decode_beam", mutant_beam(slip))
     assert failing_pins(BEAM_PINS), f"no beam pin fails with the slip '{slip}'"
+
+
+# ------------------------------------------------------------ append
+
+def mutant_append(slip):
+    """Write k_new[b] / v_new[b] at row pos[b] of copies of the caches (rows
+    outside [0, m) write nothing), with `slip` planted."""
+    def append(k_cache, v_cache, k_new, v_new, pos):
+        k_out = k_cache if slip == "in_place" else np.array(k_cache, copy=True)
+        v_out = v_cache if slip == "in_place" else np.array(v_cache, copy=True)
+        for bi, p in enumerate(int(x) for x in pos):
+            p = p + 1 if slip == "row_off_by_one" else p
+            if slip == "no_range_check" or 0 <= p < k_out.shape[1]:
+                k_out[bi, p] = k_new[bi]
+                v_out[bi, p] = v_new[bi]
+        return k_out, v_out
+    return append
+
+
+APPEND_PINS = [
+    ("append is the concat", T.test_append_is_the_concat_of_the_review),
+    ("append out of range writes nothing", T.test_append_out_of_range_row_writes_nothing),
+]
+
+
+def test_append_mutant_without_a_slip_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(T, "oracle_kv_append", mutant_append(None))
+    assert failing_pins(APPEND_PINS) == []
+
+
+@pytest.mark.parametrize("slip", ["row_off_by_one", "in_place", "no_range_check"])
+def test_an_append_pin_catches_the_planted_slip(monkeypatch, slip):
+    monkeypatch.setattr(T, "oracle_kv_append", mutant_append(slip))
+    assert failing_pins(APPEND_PINS), f"no append pin fails with the slip '{slip}'"
