@@ -4,7 +4,7 @@ import torch
 
 from grouped_query_attention_mqa_b200.workloads import (WORKLOADS, append_algorithmic_bytes, bf16_bits_to_f32,
                                                          decode_algorithmic_bytes, decode_flops, f32_to_bf16_bits,
-                                                         host_inputs)
+                                                         host_inputs, kv_cache_bytes)
 
 
 def test_bf16_rounding_matches_torch():
@@ -53,3 +53,22 @@ def test_byte_and_flop_counts():
     assert decode_flops(wl, lens) == 64 * 4608 * 32 * 2 * 256
     # MQA at h = 32: 32 FLOP per byte of K/V (the tensor-core case)
     assert decode_flops(wl, lens) / kv == 32
+
+
+def test_counts_follow_the_incremental_complexity_analysis():
+    """Study notes §5 (complexity: §5.1 incremental MHA, §5.2 incremental MQA),
+    with k = v = d/h: the MHA K+V cache is 2·b·n·h·d_h = 2·b·n·d and the MQA one
+    2·b·n·d_h = 2·b·n·d/h; every query head still computes its own scores and
+    weighted sum (h·n·d_h = n·d per sequence), so the FLOPs do not change; the
+    memory-to-arithmetic term that grows with n goes from n/d to n/(d·h)."""
+    b, n, h, dh, e = 4, 1000, 8, 16, 2
+    d = h * dh
+    assert kv_cache_bytes(b, n, h, dh, dh, e) == 2 * b * n * d * e
+    assert kv_cache_bytes(b, n, 1, dh, dh, e) * h == 2 * b * n * d * e
+    mha = WORKLOADS["mha_b16_m16k"].with_(b=b, h=h, g=h, d_k=dh, d_v=dh, m_max=n)
+    mqa = mha.with_(g=1)
+    lens = np.full(b, n)
+    assert decode_flops(mha, lens) == decode_flops(mqa, lens) == b * n * h * 2 * (dh + dh)
+    kv = lambda wl: decode_algorithmic_bytes(wl, lens) - b * h * 2 * dh * e   # drop q and o
+    assert kv(mha) == h * kv(mqa)
+    assert (kv(mha) / decode_flops(mha, lens)) / (kv(mqa) / decode_flops(mqa, lens)) == h
