@@ -72,3 +72,28 @@ def test_counts_follow_the_incremental_complexity_analysis():
     kv = lambda wl: decode_algorithmic_bytes(wl, lens) - b * h * 2 * dh * e   # drop q and o
     assert kv(mha) == h * kv(mqa)
     assert (kv(mha) / decode_flops(mha, lens)) / (kv(mqa) / decode_flops(mqa, lens)) == h
+
+
+def test_prefill_flops_count_the_attended_pairs():
+    """4·h·d FLOPs per attended (query, key) pair; the pairs are those the
+    causal mask keeps (key u <= query t), or all n² without it."""
+    from grouped_query_attention_mqa_b200.workloads import PrefillWorkload, prefill_flops
+    for causal in (True, False):
+        wl = PrefillWorkload("t", b=3, n=7, h=4, g=2, d=16, causal=causal, scale=1.0)
+        keep = np.tril(np.ones((7, 7))) if causal else np.ones((7, 7))
+        assert prefill_flops(wl) == 4 * 4 * 16 * int(keep.sum()) * 3
+
+
+def test_beam_bytes_read_the_shared_prefix_once():
+    """The beams' step moves W-1 fewer copies of each prefix than the same step
+    over caches holding the prefix once per beam (the b·W-sequence layout)."""
+    from grouped_query_attention_mqa_b200.workloads import BEAM_WORKLOADS, Workload, beam_algorithmic_bytes
+    bw = BEAM_WORKLOADS["beam4_mqa_b64_p8k"]
+    rng = np.random.default_rng(0)
+    lp = rng.integers(bw.lp_lo, bw.lp_hi + 1, size=bw.b)
+    ls = rng.integers(bw.ls_lo, bw.ls_hi + 1, size=bw.b * bw.W)
+    copied = Workload("copied", b=bw.b * bw.W, h=bw.h, g=bw.g, d_k=bw.d, d_v=bw.d, m_max=bw.m_p + bw.m_s,
+                      len_lo=1, len_hi=bw.m_p + bw.m_s, dtype="bf16", scale=bw.scale)
+    lens_copied = np.repeat(lp, bw.W) + ls
+    saved = (bw.W - 1) * int(lp.sum()) * bw.g * 2 * bw.d * 2
+    assert decode_algorithmic_bytes(copied, lens_copied) - beam_algorithmic_bytes(bw, lp, ls) == saved
