@@ -55,6 +55,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=3000)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="time the named workload only (no other workloads)")
     return p.parse_args()
 
 
@@ -270,6 +271,288 @@ def resolve_path(binding, torch, requested):
         return "simt"
 
 
+def capture_steps(torch, stream, fn, i0, n):
+    """A CUDA graph of the n steps fn(i0) .. fn(i0 + n - 1)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(i0, i0 + n):
+            fn(i)
+    return g
+
+
+class GraphSteps:
+    """Exactly K steps fn(0) .. fn(K-1), captured in CUDA graphs: one graph of
+    G = min(K, g_max) steps replayed K // G times, then one graph of the
+    K % G remaining steps.  With g_max a multiple of the rotation period of
+    fn, every step of the run uses the input that fn(i) names."""
+
+    def __init__(self, torch, stream, fn, K, g_max):
+        self.torch, self.stream, self.K = torch, stream, K
+        self.G = min(K, g_max)
+        self.R, r = divmod(K, self.G)
+        self.full = capture_steps(torch, stream, fn, 0, self.G)
+        self.rest = capture_steps(torch, stream, fn, self.R * self.G, r) if r else None
+        self.replays(1)                      # untimed: first replays upload the graphs
+        torch.cuda.synchronize()
+
+    def launch(self):
+        if self.R == 1 and self.rest is None:
+            return f"one CUDA graph of the {self.K} steps, replayed once"
+        tail = f" + one graph of {self.K - self.R * self.G} steps" if self.rest is not None else ""
+        return f"CUDA graph of {self.G} steps replayed {self.R} times{tail} (exactly {self.K} steps)"
+
+    def replays(self, n_runs):
+        with self.torch.cuda.stream(self.stream):
+            for _ in range(n_runs):
+                for _ in range(self.R):
+                    self.full.replay()
+                if self.rest is not None:
+                    self.rest.replay()
+
+    def time(self, world, burn_in_s=0.25, device_index=0):
+        """Burn-in replays (untimed, so the clock record has samples under
+        load), then the timed run of exactly K steps between CUDA events on
+        the steps' stream.  Returns (elapsed ms, clock record)."""
+        torch = self.torch
+        import torch.distributed as dist
+        clocks = ClockSampler(device_index)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < burn_in_s or n < 1:
+            self.replays(1)
+            torch.cuda.synchronize()
+            n += 1
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            start.record(self.stream)
+            self.replays(1)
+            end.record(self.stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        if clk is not None:
+            clk["window"] = f"{burn_in_s:.2f} s of the same steps replayed back to back just before the timed run, and the run"
+        if world > 1:
+            dist.barrier()
+        return start.elapsed_time(end), clk
+
+
+def launches_per_step(wl, path, window):
+    """Kernels one fused step launches: the decode, and the merge unless no
+    sequence can span two tiles (128 rows on tcgen05, 64 on the CUDA cores)."""
+    span = min(wl.m_max, window) if window > 0 else wl.m_max
+    return 1 + (span > (128 if path == "tcgen05" else 64))
+
+
+def decode_workload_entry(torch, binding, wl, K, path, world, rank, local, seed_base=SEED, g_max=1200):
+    """One fused-step workload timed like the headline (device-resident
+    inputs, rotating cache copies, exactly K steps from CUDA graphs)."""
+    from grouped_query_attention_mqa_b200.workloads import device_inputs
+    cache_bytes = wl.b * wl.m_max * wl.g * (wl.d_k + wl.d_v) * wl.elem_bytes
+    copies = max(3, min(8, -(-3 * L2_BYTES // cache_bytes) + 1))
+    inp = device_inputs(wl, seed=seed_base + rank, device="cuda", copies=copies)
+    lens_np = inp["lens"]
+    lens = torch.from_numpy(lens_np).cuda()
+    out = torch.empty((wl.b, wl.h, wl.d_v), dtype=inp["q"].dtype, device="cuda")
+    ws = binding.new_workspace(wl.b, wl.h, wl.g, wl.d_v)
+    stream = torch.cuda.Stream()
+    plans = [binding.DecodePlan(inp["q"], inp["k"][c], inp["v"][c], lens, wl.scale, out=out, workspace=ws, path=path,
+                                stream=stream, k_new=inp["k_new"], v_new=inp["v_new"]) for c in range(copies)]
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            plans[i % copies].run()
+    torch.cuda.synchronize()
+    gs = GraphSteps(torch, stream, lambda i: plans[i % copies].run(), K, g_max - g_max % copies)
+    ms, clk = gs.time(world, device_index=local)
+    ms = reduce_over_ranks([ms], "cuda")[0] / K
+    alg = decode_algorithmic_bytes(wl, lens_np) + append_algorithmic_bytes(wl)
+    peak, _ = peaks()
+    entry = {"us_per_step": 1e3 * ms, "query_tokens_per_s": world * wl.b / (ms / 1e3),
+             "achieved_gbs": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peak,
+             "algorithmic_bytes_per_step": alg, "kv_cache_bytes": cache_bytes,
+             "shape": f"b={wl.b} h={wl.h} g={wl.g} d={wl.d_k} m_max={wl.m_max} lens U[{wl.len_lo},{wl.len_hi}] "
+                      f"mean {float(lens_np.mean()):.0f}", "path": path, "steps": K, "launch": gs.launch(),
+             "l2": f"{copies} rotating cache copies", "clocks": clk}
+    del gs, plans, inp, out, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def paper_decoder_entry(torch, binding, world, rank, local, K):
+    """The paper-shaped decoder: 128 sequences, h=8, g=1, d=128, 128 fused
+    steps with the cache growing from 1 to 128 rows (all sequences equal), as
+    one CUDA graph of the 128 steps; the average step time over the growth.
+    The whole cache is 8 MiB, so it stays in L2 as it would in the pages'
+    setting."""
+    wl = WORKLOADS["paper_mqa_b128_m128"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1000 + rank)
+    rnd = lambda *s: torch.randn(s, generator=gen, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+    K_c, V_c = rnd(wl.b, wl.m_max, wl.g, wl.d_k), rnd(wl.b, wl.m_max, wl.g, wl.d_v)
+    q, kn, vn = rnd(wl.b, wl.h, wl.d_k), rnd(wl.b, wl.g, wl.d_k), rnd(wl.b, wl.g, wl.d_v)
+    T = wl.steps
+    lens = [torch.full((wl.b,), t, dtype=torch.int32, device="cuda") for t in range(1, T + 1)]
+    out = torch.empty((wl.b, wl.h, wl.d_v), dtype=torch.bfloat16, device="cuda")
+    ws = binding.new_workspace(wl.b, wl.h, wl.g, wl.d_v)
+    stream = torch.cuda.Stream()
+    plans = [binding.DecodePlan(q, K_c, V_c, lens[t], wl.scale, out=out, workspace=ws, stream=stream, k_new=kn,
+                                v_new=vn) for t in range(T)]
+    with torch.cuda.stream(stream):
+        for p in plans:
+            p.run()
+    torch.cuda.synchronize()
+    n = T * max(1, -(-K // T))               # whole growth sequences, at least K steps
+    gs = GraphSteps(torch, stream, lambda i: plans[i % T].run(), n, T * max(1, 1200 // T))
+    ms, clk = gs.time(world, device_index=local)
+    ms = reduce_over_ranks([ms], "cuda")[0] / n
+    alg = sum(decode_algorithmic_bytes(wl, np.full(wl.b, t)) for t in range(1, T + 1)) / T + append_algorithmic_bytes(wl)
+    entry = {"us_per_step": 1e3 * ms, "query_tokens_per_s": world * wl.b / (ms / 1e3),
+             "achieved_gbs": alg / (ms / 1e3) / 1e9, "bound": "latency (8 MiB cache, L2-resident)",
+             "shape": "b=128 h=8 g=1 d=128, cache grows 1..128 over 128 steps", "steps": n, "launch": gs.launch(),
+             "clocks": clk}
+    del gs, plans, K_c, V_c, out, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def beam_entry(torch, binding, wl, K, local, seed=SEED):
+    """mqa_decode_beam timed like the headline (exactly K steps from CUDA
+    graphs, two rotating copies of the prefix caches), beside the same step
+    with the prefix copied into every beam's cache (b*W sequences through
+    mqa_decode), which must agree with it."""
+    from grouped_query_attention_mqa_b200.workloads import beam_algorithmic_bytes, beam_device_inputs
+    inp = beam_device_inputs(wl, seed, "cuda")
+    lp, ls = torch.from_numpy(inp["lp"]).cuda(), torch.from_numpy(inp["ls"]).cuda()
+    copies = [(inp["pk"], inp["pv"]), (inp["pk"].clone(), inp["pv"].clone())]
+    out = torch.empty((wl.b, wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(256, binding.lib().mqa_decode_beam_workspace_size(wl.b, wl.W, wl.h, wl.g, wl.d)),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        pk, pv = copies[i % 2]
+        binding.decode_beam(inp["q"], pk, pv, lp, inp["sk"], inp["sv"], ls, wl.scale, out=out, workspace=ws,
+                            stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize()
+    gs = GraphSteps(torch, stream, step, K, 400)
+    ms, clk = gs.time(1, device_index=local)
+    ms /= K
+    launch = gs.launch()
+    del gs
+    # the same step with the prefix copied into every beam's cache (b*W independent sequences)
+    rows = wl.m_p + wl.m_s
+    rk = torch.zeros((wl.b * wl.W, rows, wl.g, wl.d), dtype=torch.bfloat16, device="cuda")
+    rv = torch.zeros_like(rk)
+    for s_ in range(wl.b):
+        for w in range(wl.W):
+            r, a, c = s_ * wl.W + w, int(inp["lp"][s_]), int(inp["ls"][s_ * wl.W + w])
+            rk[r, :a] = inp["pk"][s_, :a]
+            rv[r, :a] = inp["pv"][s_, :a]
+            rk[r, a:a + c] = inp["sk"][r, :c]
+            rv[r, a:a + c] = inp["sv"][r, :c]
+    rlens = (lp.repeat_interleave(wl.W) + ls).to(torch.int32)
+    rout = torch.empty((wl.b * wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
+    rplan = binding.DecodePlan(inp["q"].view(wl.b * wl.W, wl.h, wl.d), rk, rv, rlens, wl.scale, out=rout,
+                               stream=stream)
+    with torch.cuda.stream(stream):
+        rplan.run()
+    torch.cuda.synchronize()
+    Kr = max(3, K // 4)
+    gr = GraphSteps(torch, stream, lambda i: rplan.run(), Kr, 400)
+    ms_rep, _ = gr.time(1, burn_in_s=0.05, device_index=local)
+    ms_rep /= Kr
+    del gr
+    step(0)
+    torch.cuda.synchronize()
+    if not torch.allclose(rout.float(), out.view(wl.b * wl.W, wl.h, wl.d).float(), atol=1.5e-2, rtol=0):
+        raise RuntimeError("the shared-prefix and the replicated step disagree")
+    alg = beam_algorithmic_bytes(wl, inp["lp"], inp["ls"])
+    peak, _ = peaks()
+    tok = wl.b * wl.W
+    entry = {"us_per_step": 1e3 * ms, "query_tokens_per_s": tok / (ms / 1e3), "achieved_gbs": alg / (ms / 1e3) / 1e9,
+             "frac": alg / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": alg,
+             "shape": f"b={wl.b} beams={wl.W} h={wl.h} g={wl.g} d={wl.d} prefixes U[{wl.lp_lo},{wl.lp_hi}] "
+                      f"suffixes U[{wl.ls_lo},{wl.ls_hi}]",
+             "replicated_prefix_us_per_step": 1e3 * ms_rep, "shared_over_replicated_speedup": ms_rep / ms,
+             "steps": K, "launch": launch, "l2": "2 rotating prefix-cache copies", "clocks": clk}
+    del inp, copies, out, ws, rk, rv, rout, rplan
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def prefill_entry(torch, binding, wl, K, rank, local):
+    """mqa_prefill on packed equal-length sequences, exactly K launches from
+    CUDA graphs: TFLOP/s (4 h d FLOPs per attended pair) against the measured
+    bf16 tensor peak (burst and sustained)."""
+    from grouped_query_attention_mqa_b200.workloads import prefill_device_inputs
+    inp = prefill_device_inputs(wl, seed=rank_seed(rank), device="cuda")
+    out = torch.empty_like(inp["q"])
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        binding.prefill(inp["q"], inp["k"], inp["v"], inp["cu"], wl.n, wl.scale, causal=wl.causal, out=out,
+                        stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize()
+    gs = GraphSteps(torch, stream, step, K, 100)
+    ms, clk = gs.time(1, device_index=local)
+    ms /= K
+    flops = prefill_flops(wl)
+    tf = flops / (ms / 1e3) / 1e12
+    burst, sustained = tensor_peaks()
+    entry = {"ms_per_step": ms, "tflops": tf, "frac_of_burst_peak": tf / burst if burst else None,
+             "frac_of_sustained_peak": tf / sustained if sustained else None, "algorithmic_flops_per_step": flops,
+             "shape": f"b={wl.b} n={wl.n} h={wl.h} g={wl.g} d={wl.d} causal={wl.causal}", "steps": K,
+             "launch": gs.launch(), "clocks": clk}
+    del gs, inp, out
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def tensor_peaks():
+    """Measured dense bf16 peaks (burst, sustained) in TFLOP/s, or the
+    fallback figures when no measurement is present."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained") or p["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0
+
+
+def extra_entries(torch, binding, world, rank, local, K):
+    """The other workloads of the metric's family, each timed in this run:
+    GQA-8, the MHA/MQA pair on identical shapes, and the paper-shaped decoder;
+    then the beam step and the prefill (their own units)."""
+    ex = {}
+    for name in ("gqa8_b32_m32k", "mha_b16_m16k", "mqa_b16_m16k"):
+        wl = WORKLOADS[name]
+        ex[name] = decode_workload_entry(torch, binding, wl, K, resolve_path(binding, torch, "auto"), world, rank,
+                                         local)
+    mha, mqa = ex["mha_b16_m16k"], ex["mqa_b16_m16k"]
+    ex["mha_over_mqa"] = {"time_ratio": mha["us_per_step"] / mqa["us_per_step"],
+                          "kv_cache_bytes_ratio": mha["kv_cache_bytes"] / mqa["kv_cache_bytes"],
+                          "note": "same b, h, d and lengths; g = h = 32 against g = 1"}
+    ex["paper_mqa_b128_m128"] = paper_decoder_entry(torch, binding, world, rank, local, K)
+    ex["beam4_mqa_b64_p8k"] = beam_entry(torch, binding, BEAM_WORKLOADS["beam4_mqa_b64_p8k"], K, local)
+    ex["prefill_mqa_b8_n4096"] = prefill_entry(torch, binding, PREFILL_WORKLOADS["prefill_mqa_b8_n4096"], K, rank,
+                                               local)
+    return ex
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -312,43 +595,20 @@ def run_ours(args):
         for i in range(max(3, args.warmup)):
             steps[i % copies].run()
     torch.cuda.synchronize()
-    # A serving loop replays its steps from a CUDA graph: G steps per graph (a
-    # multiple of the cache copies, so the rotation runs on across replays).
-    G_dev = 40 * copies
-    dev_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(dev_graph, stream=stream):
-        for i in range(G_dev):
-            steps[i % copies].run()
-    with torch.cuda.stream(stream):
-        dev_graph.replay()
-    torch.cuda.synchronize()
 
-    # timed region: exactly K steps back to back (K // G graph replays, the
-    # rest launched one by one), CUDA events on the steps' stream around the
-    # whole run (events between steps would break the programmatic dependent
-    # launch between one step's merge and the next step's decode)
+    # Timed region: exactly K steps back to back, replayed from CUDA graphs as
+    # a serving loop would, CUDA events on the steps' stream around the whole
+    # run (events between steps would break the programmatic dependent launch
+    # between one step's kernels and the next step's).
     K = args.steps
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    time.sleep(0.2)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(K // G_dev):
-            dev_graph.replay()
-        for i in range(K - K % G_dev, K):
-            steps[i % copies].run()
-        end.record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    elapsed_ms = reduce_over_ranks([start.elapsed_time(end)], "cuda")[0]
+    gs = GraphSteps(torch, stream, lambda i: steps[i % copies].run(), K, 40 * copies)
+    elapsed_ms, clk = gs.time(world, device_index=local)
+    elapsed_ms = reduce_over_ranks([elapsed_ms], "cuda")[0]
     dec_avg_ms = elapsed_ms / K          # average duration of one step's launches
     ms_per_step = elapsed_ms / K
     value = job_value(world, b, K, elapsed_ms)
+    launch_desc = gs.launch()
+    del gs
 
     # End to end through the public API, pipelined the way a serving loop
     # overlaps transfers with compute: while step i runs its kernels, step
@@ -444,12 +704,21 @@ def run_ours(args):
         raise RuntimeError("pipelined end-to-end output differs from the device-resident step")
     e2e_ms = reduce_over_ranks([s2.elapsed_time(e2)], "cuda")[0]
     e2e_value = job_value(world, b, E, e2e_ms)
+    del graph, slots, steps
+    del inp
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     alg_bytes = decode_algorithmic_bytes(wl, lens_np, args.window) + append_algorithmic_bytes(wl)
     peak, peak_kind = peaks()
     achieved = alg_bytes / (dec_avg_ms / 1e3) / 1e9
     kernel = "decode_tc_kernel" if path == "tcgen05" else "decode_simt_kernel"
     traffic = recorded_traffic(kernel, wl.name, source_digest(path))
+    per_step = launches_per_step(wl, path, args.window)
+
+    extras = None
+    if args.workload == DEFAULT_WORKLOAD and not args.window and not args.no_extra:
+        extras = extra_entries(torch, binding, world, rank, local, K)
 
     line = None
     if rank == 0:
@@ -468,20 +737,23 @@ def run_ours(args):
                        "l2": f"{copies} rotating K/V cache copies ({copies * cache_bytes / 2**20:.0f} MiB) so each "
                              f"step's rows were evicted by >= 2 other steps' reads",
                        "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)",
-                       "launch": f"CUDA graphs of {G_dev} steps replayed back to back",
+                       "launch": launch_desc,
                        **({"window": args.window} if args.window else {})},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": f"one step = mqa_decode_append call ({kernel} + merge_kernel), average over "
-                                   f"the {K} timed steps",
+                         "kernel": f"one step = mqa_decode_append call ({kernel}"
+                                   + (" + merge_kernel" if per_step > 1 else "") + f"), average over the {K} "
+                                   "timed steps",
                          "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": dec_avg_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": E, "pipeline": f"2 slots; one staging copy in, kernels, output out, on three streams; CUDA graph of "
                                             f"{G} steps replayed {R} times"},
-            "gpu_launches": 2 * K,
+            "gpu_launches": per_step * K,
             "clocks": clk,
         }
+        if extras is not None:
+            line["workloads"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -555,34 +827,16 @@ def run_prefill(args):
     if not os.path.exists(LIB):
         build()
     binding.load_library()
-    inp = prefill_device_inputs(wl, seed=rank_seed(rank), device="cuda")
-    out = torch.empty_like(inp["q"])
-    flops = prefill_flops(wl)
-
-    def step():
-        binding.prefill(inp["q"], inp["k"], inp["v"], inp["cu"], wl.n, wl.scale, causal=wl.causal, out=out)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
     K = args.steps
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    clocks = ClockSampler(local)
-    time.sleep(0.2)
-    start.record()
-    for _ in range(K):
-        step()
-    end.record()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    elapsed_ms = reduce_over_ranks([start.elapsed_time(end)], "cuda")[0]
-    ms = elapsed_ms / K
+    ent = prefill_entry(torch, binding, wl, K, rank, local)
+    ms = reduce_over_ranks([ent["ms_per_step"]], "cuda")[0]
+    flops = prefill_flops(wl)
     tflops = flops / (ms / 1e3) / 1e12
     value = tflops * world
 
     # end to end: q, k, v copied in from pinned host memory and o copied out, every step
+    inp = prefill_device_inputs(wl, seed=rank_seed(rank), device="cuda")
+    out = torch.empty_like(inp["q"])
     host = {name: inp[name].cpu().pin_memory() for name in ("q", "k", "v")}
     o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     dev_in = {name: torch.empty_like(inp[name]) for name in ("q", "k", "v")}
@@ -599,13 +853,8 @@ def run_prefill(args):
     e2e_ms = reduce_over_ranks([s2.elapsed_time(e2)], "cuda")[0] / E
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o_h.numel() * o_h.element_size()
-    pk = None
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
-            pk = json.load(fh).get("bf16_tflops")
-    except OSError:
-        pass
-    peak, peak_kind = (float(pk), "measured") if pk else (1590.0, "fallback")
+    burst, sustained = tensor_peaks()
+    peak_kind = "measured" if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else "fallback"
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -619,17 +868,18 @@ def run_prefill(args):
             "config": {"workload": wl.name, "b": wl.b, "n": wl.n, "h": wl.h, "g": wl.g, "d": wl.d,
                        "causal": wl.causal, "tokens_per_s": wl.total * world / (ms / 1e3),
                        "l2": "q and o (2 x %d MiB) exceed the L2; K/V tiles are meant to be reused from it"
-                             % (inp["q"].numel() * 2 // 2**20),
+                             % (inp["q"].numel() * 2 // 2**20), "launch": ent["launch"],
                        "parallelism": f"replicated per GPU x{world} (independent sequences, no collective)"},
-            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": tflops / peak, "traffic": None, "peak_kind": peak_kind,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": burst, "unit": "TFLOP/s",
+                         "frac": tflops / burst, "frac_of_sustained": tflops / sustained, "traffic": None,
+                         "peak_kind": peak_kind,
                          "kernel": "prefill_tc_kernel, average over the timed steps",
                          "algorithmic_flops_per_launch": flops, "launch_ms": ms},
             "cpu_baseline": cpu,
             "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E},
             "gpu_launches": K,
-            "clocks": clk,
+            "clocks": ent["clocks"],
         }), flush=True)
     if world > 1:
         dist.barrier()
@@ -677,55 +927,20 @@ def run_beam(args):
                           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
               flush=True)
         return
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if not os.path.exists(LIB):
         build()
     binding.load_library()
+    K = args.steps
+    ent = beam_entry(torch, binding, wl, K, local)
+    ms = ent["us_per_step"] / 1e3
+    # end to end: q in from pinned host memory and o out, every step
     inp = beam_device_inputs(wl, SEED, "cuda")
     lp, ls = torch.from_numpy(inp["lp"]).cuda(), torch.from_numpy(inp["ls"]).cuda()
     out = torch.empty((wl.b, wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(binding.lib().mqa_decode_beam_workspace_size(wl.b, wl.W, wl.h, wl.g, wl.d), dtype=torch.uint8,
-                     device="cuda")
-
-    def step():
-        binding.decode_beam(inp["q"], inp["pk"], inp["pv"], lp, inp["sk"], inp["sv"], ls, wl.scale, out=out,
-                            workspace=ws)
-
-    def timed(fn, K):
-        for _ in range(max(3, args.warmup)):
-            fn()
-        torch.cuda.synchronize()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
-        for _ in range(K):
-            fn()
-        s1.record()
-        torch.cuda.synchronize()
-        return s0.elapsed_time(s1) / K
-
-    K = args.steps
-    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
-    time.sleep(0.2)
-    ms = timed(step, K)
-    clk = clocks.stop()
-    # the same step with the prefix copied into every beam's cache (b*W independent sequences)
-    rows = wl.m_p + wl.m_s
-    rk = torch.zeros((wl.b * wl.W, rows, wl.g, wl.d), dtype=torch.bfloat16, device="cuda")
-    rv = torch.zeros_like(rk)
-    for s_ in range(wl.b):
-        for w in range(wl.W):
-            r, a, c = s_ * wl.W + w, int(inp["lp"][s_]), int(inp["ls"][s_ * wl.W + w])
-            rk[r, :a] = inp["pk"][s_, :a]
-            rv[r, :a] = inp["pv"][s_, :a]
-            rk[r, a:a + c] = inp["sk"][r, :c]
-            rv[r, a:a + c] = inp["sv"][r, :c]
-    rlens = (lp.repeat_interleave(wl.W) + ls).to(torch.int32)
-    rout = torch.empty((wl.b * wl.W, wl.h, wl.d), dtype=torch.bfloat16, device="cuda")
-    rplan = binding.DecodePlan(inp["q"].view(wl.b * wl.W, wl.h, wl.d), rk, rv, rlens, wl.scale, out=rout)
-    ms_rep = timed(rplan.run, max(10, K // 4))
-    if not torch.allclose(rout.float(), out.view(wl.b * wl.W, wl.h, wl.d).float(), atol=1.5e-2, rtol=0):
-        raise RuntimeError("the shared-prefix and the replicated step disagree")
-    # end to end: q in from pinned host memory and o out, every step
+    ws = torch.empty(max(256, binding.lib().mqa_decode_beam_workspace_size(wl.b, wl.W, wl.h, wl.g, wl.d)),
+                     dtype=torch.uint8, device="cuda")
     q_h = inp["q"].cpu().pin_memory()
     o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     q_d = torch.empty_like(inp["q"])
@@ -735,10 +950,18 @@ def run_beam(args):
         binding.decode_beam(q_d, inp["pk"], inp["pv"], lp, inp["sk"], inp["sv"], ls, wl.scale, out=out, workspace=ws)
         o_h.copy_(out, non_blocking=True)
 
-    e2e_ms = timed(e2e_step, max(10, K // 4))
-    alg = beam_algorithmic_bytes(wl, inp["lp"], inp["ls"])
+    E = max(10, K // 4)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(E):
+        e2e_step()
+    s1.record()
+    torch.cuda.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / E
     peak, peak_kind = peaks()
-    achieved = alg / (ms / 1e3) / 1e9
     tok = wl.b * wl.W
     print(json.dumps({
         "metric": BEAM_METRIC, "value": tok / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K,
@@ -746,19 +969,19 @@ def run_beam(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "b": wl.b, "beams": wl.W, "h": wl.h, "g": wl.g, "d": wl.d,
                    "prefix_lens": f"U[{wl.lp_lo},{wl.lp_hi}]", "suffix_lens": f"U[{wl.ls_lo},{wl.ls_hi}]",
-                   "replicated_prefix_ms_per_step": ms_rep,
-                   "replicated_prefix_query_tokens_per_s": tok / (ms_rep / 1e3),
-                   "l2": "the prefix caches exceed the L2 (%d MiB)" % (inp["pk"].numel() * 4 // 2**20)},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_kind": peak_kind,
+                   "replicated_prefix_ms_per_step": ent["replicated_prefix_us_per_step"] / 1e3,
+                   "replicated_prefix_query_tokens_per_s": tok / (ent["replicated_prefix_us_per_step"] / 1e6),
+                   "launch": ent["launch"], "l2": ent["l2"]},
+        "roofline": {"bound": "hbm", "achieved": ent["achieved_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": ent["frac"], "traffic": None, "peak_kind": peak_kind,
                      "kernel": "one step = decode_tc_beam_kernel (prefix once for the W beams, then each beam's "
-                               "suffix) + merge_kernel", "algorithmic_bytes_per_launch": alg,
+                               "suffix) + merge_kernel", "algorithmic_bytes_per_launch": ent["algorithmic_bytes_per_step"],
                      "launch_ms": ms},
         "cpu_baseline": None,
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": q_h.numel() * 2,
-                "d2h_bytes_per_step": o_h.numel() * 2, "steps": max(10, K // 4)},
-        "gpu_launches": 3 * K,
-        "clocks": clk,
+                "d2h_bytes_per_step": o_h.numel() * 2, "steps": E},
+        "gpu_launches": 2 * K,
+        "clocks": ent["clocks"],
     }), flush=True)
 
 
