@@ -14,7 +14,7 @@ from grouped_query_attention_mqa_b200.build import build
 from grouped_query_attention_mqa_b200.workloads import WORKLOADS, Workload, bf16_bits_to_f32, device_inputs, host_inputs
 from oracle import oracle_decode, oracle_decode_step, oracle_kv_append
 
-from gpu_util import assert_close, bits, dev, host64
+from gpu_util import assert_close, bits, check_full_size_step, dev, host64
 
 pytestmark = pytest.mark.gpu
 
@@ -104,26 +104,17 @@ def test_paper_decoder_128_fused_steps(path):
     assert np.array_equal(bits(Kd), K_host) and np.array_equal(bits(Vd), V_host)
 
 
-@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k"])
-def test_full_size_fused_step_sampled(name):
-    """The bench's step on the full-size workloads; sampled sequences against
-    the oracle from copies of their rows taken before the step."""
+@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k", "mqa_b16_m16k", "mha_b16_m16k"])
+def test_full_size_fused_step_every_sequence(name):
+    """The bench's step (mqa_decode_append, default path and CTA count) on the
+    full-size workloads; every sequence against the oracle, and the caches:
+    old rows untouched, row lens-1 the step's new row."""
     wl = WORKLOADS[name]
     inp = device_inputs(wl, seed=4, device="cuda")
     lens = inp["lens"]
     K, V = inp["k"][0], inp["v"][0]
-    picks = sorted({0, len(lens) - 1, int(np.argmax(lens)), int(np.argmin(lens)), len(lens) // 2})
-    before = {bi: (K[bi, : lens[bi]].float().cpu().numpy(), V[bi, : lens[bi]].float().cpu().numpy()) for bi in picks}
-    o = host64(binding.decode_append(inp["q"], K, V, inp["k_new"], inp["v_new"], torch.from_numpy(lens).cuda(),
-                                     wl.scale))
-    assert np.isfinite(o).all()
-    qf, knf, vnf = (inp[x].float().cpu().numpy() for x in ("q", "k_new", "v_new"))
-    for bi in picks:
-        Kb, Vb = before[bi]
-        ref, _, _, _ = oracle_decode_step(qf[bi:bi + 1], Kb[None], Vb[None], knf[bi:bi + 1], vnf[bi:bi + 1],
-                                          np.array([lens[bi] - 1]), wl.g, wl.scale)
-        assert_close(o[bi:bi + 1], ref, wl.dtype, f"{name} seq {bi}")
-        assert torch.equal(K[bi, lens[bi] - 1].view(torch.int16), inp["k_new"][bi].reshape(-1).view(torch.int16)
-                           .reshape(K[bi, lens[bi] - 1].shape))
-    del inp, K, V
+    o = binding.decode_append(inp["q"], K, V, inp["k_new"], inp["v_new"], torch.from_numpy(lens).cuda(), wl.scale)
+    torch.cuda.synchronize()
+    check_full_size_step(o, wl, 4, lens, name, K, V, inp["k_new"], inp["v_new"])
+    del inp, K, V, o
     torch.cuda.empty_cache()

@@ -112,3 +112,31 @@ def test_prefill_empty_batch_is_a_no_op():
     q = torch.zeros((0, 8, D), dtype=torch.bfloat16, device="cuda")
     o = binding.prefill(q, q[:, :1], q[:, :1], torch.zeros(1, dtype=torch.int32, device="cuda"), 0, 1.0)
     assert o.shape == (0, 8, D)
+
+
+@pytest.mark.parametrize("name", ["prefill_mqa_b8_n4096", "prefill_gqa8_b4_n8192"])
+def test_prefill_bench_sizes_sampled(name):
+    """The bench's prefill workloads at full size, in the launch the bench
+    times: per sequence, positions in the first and in the last query tile
+    (the end of the sequence included), at 128-key tile edges and at random,
+    each against the decode oracle over its causal prefix."""
+    from grouped_query_attention_mqa_b200.workloads import PREFILL_WORKLOADS, prefill_device_inputs
+    wl = PREFILL_WORKLOADS[name]
+    inp = prefill_device_inputs(wl, seed=5, device="cuda")
+    o = binding.prefill(inp["q"], inp["k"], inp["v"], inp["cu"], wl.n, wl.scale, causal=wl.causal)
+    torch.cuda.synchronize()
+    kf = inp["k"].float().cpu().numpy()
+    vf = inp["v"].float().cpu().numpy()
+    rng = np.random.default_rng(17)
+    n = wl.n
+    rows_per_tile = 128 // (wl.h // wl.g)       # positions per 128-row query tile of one K/V group
+    for si in range(wl.b):
+        a = si * n
+        picks = {0, 1, rows_per_tile - 1, 127, 128, n - rows_per_tile, n - 2, n - 1}
+        picks |= set(rng.integers(0, n, size=6).tolist())
+        for t in sorted(p for p in picks if 0 <= p < n):
+            qt = inp["q"][a + t].float().cpu().numpy()[None]
+            ref, _ = oracle_decode(qt, kf[a:a + t + 1][None], vf[a:a + t + 1][None], [t + 1], wl.g, wl.scale)
+            assert_close(host64(o[a + t])[None], ref, "bf16", f"{name} seq {si} pos {t}")
+    del inp, o
+    torch.cuda.empty_cache()
