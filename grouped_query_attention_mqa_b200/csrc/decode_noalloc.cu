@@ -13,6 +13,7 @@
 // address, so the host looks the address up once per device with
 // cudaGetSymbolAddress (with that device current) and passes it to the
 // kernels like any other workspace pointer.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -26,15 +27,18 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MQA_NOALLOC_SCR
 constexpr int kMaxDevices = 64;
 
 // Device address of g_noalloc_scratch on the current device, looked up on
-// the first call per device.  Returns nullptr if the lookup fails.
+// the first call per device.  Returns nullptr if the lookup fails.  Host
+// threads may make their first calls concurrently: each slot is an atomic,
+// and two threads that both look the address up store the same value.
 void* scratch_address() {
-  static void* addr[kMaxDevices] = {nullptr};
+  static std::atomic<void*> addr[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (addr[dev] != nullptr) return addr[dev];
+  void* cached = addr[dev].load(std::memory_order_acquire);
+  if (cached != nullptr) return cached;
   void* ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-  addr[dev] = ptr;
+  addr[dev].store(ptr, std::memory_order_release);
   return ptr;
 }
 
@@ -121,7 +125,9 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.window = 0;
   a.q_beams = 0;
   a.q_group_heads = hq;
-  a.no_merge = 0;
+  // As in mqa_decode: when no sequence can span two tiles no segment is split,
+  // the decode writes every output row itself and the merge is not launched.
+  a.no_merge = m_max <= (use_tc ? tc_tile_rows() : simt_tile_rows());
   a.sk = nullptr;
   a.sv = nullptr;
   a.slens = nullptr;
@@ -132,6 +138,6 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.grid = grid;
   cudaError_t e = use_tc ? launch_decode_tc(a, stream) : launch_decode_simt(a, d_k, dtype, stream);
   if (e != cudaSuccess) return MQA_ERR_CUDA;
-  if (launch_merge(a, dtype, stream) != cudaSuccess) return MQA_ERR_CUDA;
+  if (!a.no_merge && launch_merge(a, dtype, stream) != cudaSuccess) return MQA_ERR_CUDA;
   return MQA_OK;
 }

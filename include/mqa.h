@@ -218,7 +218,11 @@ MQA_API mqa_status_t mqa_decode_append(void* o, const void* q, void* k_cache, vo
  * workspace pair; the caller still provides o, q, the caches and lens.
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current).  Make that first call before any
- *    stream capture on the device.
+ *    stream capture on the device.  Under lazy module loading (the default
+ *    since CUDA 12) that first call may also be what loads the library's
+ *    device code on the device, which reserves the 16 MiB array there; if
+ *    the device has no room left, the call returns MQA_ERR_CUDA.  A caller
+ *    that wants no surprise later makes one warm-up call at start-up.
  *  - The array holds the partials of the last call; every value a call reads
  *    back from it was written earlier in the same call, so nothing in it has
  *    to start at zero.

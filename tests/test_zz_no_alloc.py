@@ -19,7 +19,9 @@ from grouped_query_attention_mqa_b200 import binding
 from grouped_query_attention_mqa_b200.build import build
 from grouped_query_attention_mqa_b200.workloads import Workload, host_inputs
 
-from gpu_util import TOL, dev, host64
+from oracle import oracle_decode
+
+from gpu_util import TOL, assert_close, dev, host64
 
 pytestmark = pytest.mark.gpu
 
@@ -34,8 +36,9 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _both(lib, wl, seed):
-    """Run mqa_decode (caller workspace) and mqa_decode_noalloc on one input."""
+def _both(lib, wl, seed, with_oracle=False):
+    """Run mqa_decode (caller workspace) and mqa_decode_noalloc on one input;
+    with_oracle also returns the oracle's output on the same input."""
     inp = host_inputs(wl, seed, nan_tail=True)
     q, K, V = dev(inp["q"], wl.dtype), dev(inp["k"], wl.dtype), dev(inp["v"], wl.dtype)
     lens = torch.from_numpy(inp["lens"]).cuda()
@@ -51,6 +54,9 @@ def _both(lib, wl, seed):
                                 wl.d_v, wl.scale, dt, None, stream)
     assert st == binding.MQA_OK
     torch.cuda.synchronize()
+    if with_oracle:
+        want, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], inp["lens"], wl.g, wl.scale)
+        return host64(out), host64(ref), want
     return host64(out), host64(ref)
 
 
@@ -65,10 +71,40 @@ CASES = [
 @pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
 def test_noalloc_matches_decode_on_two_calls_in_a_row(lib, wl):
     for seed in (11, 12):   # second call: new inputs over the array the first call left behind
-        out, ref = _both(lib, wl, seed)
+        out, ref, want = _both(lib, wl, seed, with_oracle=True)
         assert np.isfinite(out).all()
         err = float(np.abs(out - ref).max())
         assert err <= TOL[wl.dtype], f"{wl.name} seed {seed}: max-abs {err:.3e}"
+        assert_close(out, want, wl.dtype, f"{wl.name} seed {seed} against the oracle")
+
+
+def test_noalloc_lowers_its_cta_count_to_fit_the_array(lib):
+    """960 sequences with 32 heads: each split partial takes 32 x 129 floats,
+    so only about 1000 slots fit the 16 MiB array next to the 960 segments and
+    the call runs on far fewer CTAs than the GPU has SMs.  Every sequence is
+    checked against the oracle and against mqa_decode, on two calls in a
+    row."""
+    wl = Workload("noalloc_lowered", b=960, h=32, g=1, d_k=128, d_v=128, m_max=300, len_lo=1, len_hi=300,
+                  dtype="bf16", scale=1 / math.sqrt(128))
+    per_slot = 32 * 4 + 32 * 128 * 4
+    assert (binding.MQA_NOALLOC_SCRATCH_BYTES - wl.b * 8) // per_slot - wl.b < torch.cuda.get_device_properties(
+        0).multi_processor_count
+    for seed in (21, 22):
+        out, ref, want = _both(lib, wl, seed, with_oracle=True)
+        assert_close(out, want, "bf16", f"lowered grid seed {seed} against the oracle")
+        err = float(np.abs(out - ref).max())
+        assert err <= TOL["bf16"], f"lowered grid seed {seed}: max-abs {err:.3e} against mqa_decode"
+
+
+def test_noalloc_single_tile_caches_skip_the_merge(lib):
+    """Caches of at most one tile: no sequence is split, the decode writes
+    every row itself (zero rows for empty sequences included)."""
+    wl = Workload("noalloc_short", b=40, h=16, g=2, d_k=128, d_v=128, m_max=128, len_lo=0, len_hi=128,
+                  dtype="bf16", scale=1 / math.sqrt(128))
+    for seed in (31, 32):
+        out, ref, want = _both(lib, wl, seed, with_oracle=True)
+        assert_close(out, want, "bf16", f"single-tile seed {seed} against the oracle")
+        assert np.array_equal(out, ref)
 
 
 def test_noalloc_rejects_shapes_beyond_its_array(lib):
