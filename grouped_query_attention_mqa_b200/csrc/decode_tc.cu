@@ -41,8 +41,11 @@
 //                       L2 evict-first: each byte is read once.  The two
 //                       producers sit in different warps because the waits of
 //                       two diverged threads of one warp are serialised.
-//   warp 1, lane 0      MMA issuer: S(i+1) = K Q^T while P(i) is being made,
-//                       then O += V^T P(i); completions are signalled with
+//   warp 1, lane 0      S issuer: S(i) = K Q^T into a double buffer in tensor
+//                       memory, as soon as K(i) has landed and the softmax
+//                       warps hold S(i-2) in registers.
+//   warp 11, lane 0     P.V issuer: O += V^T P(i) once P(i) is written; the two
+//                       issuers' completions are signalled with
 //                       tcgen05.commit on mbarriers.
 //   warps 2-9           softmax and epilogue in two column groups of four
 //                       warps: one cache row (then one output column) and
@@ -70,8 +73,10 @@ using namespace sm100;
 
 constexpr int kTile = 128;                   // cache rows per tile (the MMA M)
 constexpr int kD = 128;                      // head size
-constexpr int kThreads = 352;                // warp 0 K/Q loads, warp 1 MMA, warps 2-9 softmax, warp 10 V loads
+constexpr int kThreads = 384;                // warp 0 K/Q loads, warp 1 S products, warps 2-9 softmax, warp 10 V loads,
+                                             // warp 11 P.V products
 constexpr int kVWarp = 10;
+constexpr int kPvWarp = 11;
 constexpr int kNpv = 64;                     // N of the P.V product (P padded with zero columns)
 constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte swizzle column
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
@@ -87,8 +92,8 @@ template <int NP, int SK, int SV>
 struct TcCfg {
   // barriers
   static constexpr int kKFull = 0, kKEmpty = SK, kVFull = 2 * SK, kVEmpty = 2 * SK + SV, kSFull = 2 * SK + 2 * SV,
-                       kPFull = kSFull + 2, kOFull = kPFull + 1, kQFull = kOFull + 1, kQEmpty = kQFull + 2,
-                       kOFree = kQEmpty + 2, kDone = kOFree + 2, kNumBars = kDone + 1;
+                       kSEmpty = kSFull + 2, kPFull = kSEmpty + 2, kOFull = kPFull + 1, kQFull = kOFull + 1,
+                       kQEmpty = kQFull + 2, kOFree = kQEmpty + 2, kDone = kOFree + 2, kNumBars = kDone + 1;
   // shared memory
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + SK * kTileBytes;
@@ -465,99 +470,94 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
       mbar_wait(bar(C::kQFull + (sq & 1)), uint32_t(sq >> 1) & 1, kTimeoutNs);
 }
 
-// One thread issues every tensor-core product.  S(j) = K Q^T may run once
-// K(j) has landed (and, for a segment's first tile, its Q) and S buffer j&1 is
-// free, i.e. P(j-2) has been consumed; O += V^T P(j) once P(j) is written and
-// V(j) has landed.  The two streams are independent, so the thread polls both
-// and issues whichever is ready: a late K tile never holds up a P.V product
-// the softmax warps are waiting for.
+// Two threads issue the tensor-core products, each in a warp of its own: one
+// the S = K Q^T stream, one the O += V^T P stream.  A thread issuing
+// tcgen05.mma spends tens of cycles on each instruction and more on noticing
+// the event that enables it, so one thread serving both streams set the tile
+// period by itself; split, the P.V chain the softmax waits on only carries its
+// own products.  tcgen05.commit tracks the products of the committing thread,
+// so each stream releases its own ring stages.
+//
+// S(j) needs K(j) landed, for a segment's first tile its Q, and S buffer j&1
+// free: the softmax warps arrive on SEmpty once they hold S(j-2) in registers.
 template <int NP, int SK, int SV, bool kFB>
-__device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
+__device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
   using C = TcCfg<NP, SK, SV>;
   const Sched& sc = ws.s;
-  auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
-  const int64_t n = sc.t_end - sc.t_begin;
-  TileWalk<kFB> wq(a, ws, r), wp(a, ws, r);   // walkers for the S stream and the O stream
-  const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);           // K-major, rows of 128 B
+  const int n = int(sc.t_end - sc.t_begin);   // tiles of this CTA (fewer than 2^31)
+  TileWalk<kFB> w(a, ws, r);
+  const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);   // K-major, rows of 128 B
   const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
-  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
-  const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);   // MN-major P
-
-  int64_t iq = 0, ip = 0;          // next S and next O product
-  bool q_walked = false, p_walked = false;
-  uint64_t idle_since = 0;
-  uint32_t idle_polls = 0;
-  while (ip < n) {
-    bool progressed = false;
-    // S(iq): needs K(iq), Q of its segment, and P(iq-2) consumed (iq <= ip + 1)
-    if (iq < n && iq <= ip + 1) {
-      if (!q_walked) {
-        wq.next(a, sc);
-        q_walked = true;
-      }
-      const int st = int(iq % SK);
-      const int qb = wq.sidx & 1;
-      if ((!wq.first || mbar_test(bar(C::kQFull + qb), uint32_t(wq.sidx >> 1) & 1)) &&
-          mbar_test(bar(C::kKFull + st), uint32_t(iq / SK) & 1)) {
-        tc_fence_after();
-        // descriptors differ only in their start address (bits 0-13, 16-byte units)
-        const uint64_t ka = kdesc0 + ((st * kTileBytes) >> 4);
-        const uint64_t qa = qdesc0 + ((qb * C::kQBytes) >> 4);
-        const uint32_t d = r.tmem + uint32_t(iq & 1) * NP;
+  const uint32_t bar0 = r.sbase + C::kBar;
+  auto bar = [&](int id) { return bar0 + 8u * uint32_t(id); };
+  int kst = 0;
+  uint32_t kph = 0;   // ring stage of K(i) and the parity of its full barrier
+  for (int i = 0; i < n; ++i) {
+    w.next(a, sc);
+    const int qb = w.sidx & 1;
+    if (w.first && !wait_bar(r, bar(C::kQFull + qb), uint32_t(w.sidx >> 1) & 1)) break;
+    if (!wait_bar(r, bar(C::kKFull + kst), kph)) break;
+    if (i >= 2 && !wait_bar(r, bar(C::kSEmpty + (i & 1)), uint32_t((i >> 1) - 1) & 1)) break;
+    tc_fence_after();
+    // descriptors differ only in their start address (bits 0-13, 16-byte units)
+    const uint64_t ka = kdesc0 + uint64_t((uint32_t(kst) * kTileBytes) >> 4);
+    const uint64_t qa = qdesc0 + uint64_t((uint32_t(qb) * C::kQBytes) >> 4);
+    const uint32_t d = r.tmem + uint32_t(i & 1) * NP;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
-        }
-        mma_commit(bar(C::kSFull + (iq & 1)));
-        mma_commit(bar(C::kKEmpty + st));
-        if (wq.last) mma_commit(bar(C::kQEmpty + qb));
-        ++iq;
-        q_walked = false;
-        progressed = true;
-      }
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+      const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
+      mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
     }
-    // O += V^T P(ip): needs P(ip), V(ip) and, for a segment's first tile, its O buffer
-    if (ip < iq) {
-      if (!p_walked) {
-        wp.next(a, sc);
-        p_walked = true;
-      }
-      const int st = int(ip % SV);
-      const int ob = wp.sidx & 1;
-      if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) && mbar_test(bar(C::kVFull + st), uint32_t(ip / SV) & 1) &&
-          (!wp.first || wp.sidx < 2 || mbar_test(bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))) {
-        tc_fence_after();
-        const uint64_t va = vdesc0 + ((st * kTileBytes) >> 4);
-        const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
-        const uint32_t acc0 = wp.first ? 0u : 1u;
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-        mma_commit(bar(C::kOFull));
-        mma_commit(bar(C::kVEmpty + st));
-        ++ip;
-        p_walked = false;
-        progressed = true;
-      }
-    }
-    if (progressed) {
-      idle_polls = 0;
-    } else if ((++idle_polls & 1023u) == 0) {   // bounded: give up after the timeout without progress
-      const uint64_t now = globaltimer_ns();
-      if (idle_polls == 1024) {
-        idle_since = now;
-      } else if (now - idle_since > kTimeoutNs || *r.abort) {
-        *r.abort = 1;
-        set_flag(r.flags, MQA_FLAG_PIPE_TIMEOUT);
-        break;
-      }
+    mma_commit(bar(C::kSFull + (i & 1)));
+    mma_commit(bar(C::kKEmpty + kst));
+    if (w.last) mma_commit(bar(C::kQEmpty + qb));
+    if (++kst == SK) {
+      kst = 0;
+      kph ^= 1u;
     }
   }
-  // every MMA issued above has completed before tensor memory is released
+  // every product issued above has completed before tensor memory is released
+  mma_commit(bar(C::kDone));
+  mbar_wait(bar(C::kDone), 0, kTimeoutNs);
+}
+
+// O += V^T P(j) needs P(j) written, V(j) landed and, for a segment's first
+// tile, its O buffer released by the epilogue of the segment two back.
+template <int NP, int SK, int SV, bool kFB>
+__device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
+  using C = TcCfg<NP, SK, SV>;
+  const Sched& sc = ws.s;
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
+  const int n = int(sc.t_end - sc.t_begin);
+  TileWalk<kFB> w(a, ws, r);
+  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
+  const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);   // MN-major P
+  const uint32_t bar0 = r.sbase + C::kBar;
+  auto bar = [&](int id) { return bar0 + 8u * uint32_t(id); };
+  int vst = 0;
+  uint32_t vph = 0;   // ring stage of V(i) and the parity of its full barrier
+  for (int i = 0; i < n; ++i) {
+    w.next(a, sc);
+    const int ob = w.sidx & 1;
+    if (!wait_bar(r, bar(C::kPFull), uint32_t(i & 1))) break;
+    if (!wait_bar(r, bar(C::kVFull + vst), vph)) break;
+    if (w.first && w.sidx >= 2 && !wait_bar(r, bar(C::kOFree + ob), uint32_t((w.sidx >> 1) - 1) & 1)) break;
+    tc_fence_after();
+    const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * kTileBytes) >> 4);
+    const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
+    const uint32_t acc0 = w.first ? 0u : 1u;
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+    mma_commit(bar(C::kOFull));
+    mma_commit(bar(C::kVEmpty + vst));
+    if (++vst == SV) {
+      vst = 0;
+      vph ^= 1u;
+    }
+  }
   mma_commit(bar(C::kDone));
   mbar_wait(bar(C::kDone), 0, kTimeoutNs);
 }
@@ -665,6 +665,8 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     tc_fence_after();
     const bool valid = row < w.tc.rows;
     tmem_ld<CPT>(t_lane + uint32_t(i & 1) * NP + col0, sv);
+    tc_fence_before();
+    mbar_arrive(bar(C::kSEmpty + (i & 1)));   // S buffer i&1 may take S(i+2)
 #pragma unroll
     for (int k = 0; k < CPT; ++k) sv[k] = valid ? sv[k] * c : -INFINITY;
     if constexpr (kFB) {
@@ -720,6 +722,23 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 #pragma unroll
       for (int k = 0; k < CPT; ++k) mr[k] = mref[col0 + k];
     }
+    // P = exp2(s - m) in bf16, into registers before waiting for the previous
+    // product: only the shared-memory store has to follow that wait.
+    if (full && !w.first) {
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) lpart[k] *= alpha[col0 + k];
+    }
+    uint32_t packed[CPT / 2];
+#pragma unroll
+    for (int k2 = 0; k2 < CPT / 2; ++k2) {
+      const int k = 2 * k2;
+      const float p0 = col0 + k < hq ? ex2_approx(sv[k] - mr[k]) : 0.f;
+      const float p1 = col0 + k + 1 < hq ? ex2_approx(sv[k + 1] - mr[k + 1]) : 0.f;
+      lpart[k] += p0;
+      lpart[k + 1] += p1;
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+      packed[k2] = *reinterpret_cast<uint32_t*>(&b2);
+    }
     // O(i-1) must be complete before O is rescaled and before P(i) overwrites
     // the P buffer it read; a ragged tile needs its V rows landed before the
     // rows past the sequence end are zeroed.
@@ -732,44 +751,23 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     if (w.tc.rows < kTile) ok2 = wait(C::kVFull + st, uint32_t(i / SV) & 1) && ok2;
     if (!softmax_barrier_and(ok && ok2)) { failed = true; break; }
     tc_fence_after();
-    if (pend.on) {
-      epilogue(pend);
-      pend.on = false;
-    }
     if (full && !w.first) {
-      float al[CPT];
-#pragma unroll
-      for (int k = 0; k < CPT; ++k) {
-        al[k] = alpha[col0 + k];
-        lpart[k] *= al[k];
-      }
       // rescale the O accumulated so far (thread = output column, its heads)
       const uint32_t oc = t_lane + kOCol + uint32_t(w.sidx & 1) * kNpv + col0;
       float v[CPT];
       tmem_ld<CPT>(oc, v);
 #pragma unroll
-      for (int k = 0; k < CPT; ++k) v[k] *= al[k];
+      for (int k = 0; k < CPT; ++k) v[k] *= alpha[col0 + k];
       tmem_st<CPT>(oc, v);
       tmem_wait_st();
     }
-    // P = exp2(s - m), bf16, into the MN-major 128-byte-swizzled P buffer
+    // P into the MN-major 128-byte-swizzled P buffer
     unsigned char* prow = r.smem + C::kP + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
     for (int c8 = 0; c8 < CPT / 8; ++c8) {
-      uint32_t packed[4];
-#pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2) {
-        const int k = c8 * 8 + k2 * 2;
-        const float p0 = col0 + k < hq ? ex2_approx(sv[k] - mr[k]) : 0.f;
-        const float p1 = col0 + k + 1 < hq ? ex2_approx(sv[k + 1] - mr[k + 1]) : 0.f;
-        lpart[k] += p0;
-        lpart[k + 1] += p1;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        packed[k2] = *reinterpret_cast<uint32_t*>(&b2);
-      }
       const int chunk = col0 / 8 + c8;
       *reinterpret_cast<uint4*>(prow + ((chunk ^ (row & 7)) << 4)) =
-          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          make_uint4(packed[c8 * 4], packed[c8 * 4 + 1], packed[c8 * 4 + 2], packed[c8 * 4 + 3]);
     }
     if (w.tc.rows < kTile) {
       // rows past the sequence end were loaded too; zero them in V so that
@@ -786,6 +784,13 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(bar(C::kPFull));
+    // The previous segment's output, now off the path to the next product: its
+    // O buffer is final (its last product completed before the wait above) and
+    // P.V(i) accumulates into the other buffer.
+    if (pend.on) {
+      epilogue(pend);
+      pend.on = false;
+    }
 
     if (w.last) {
       // per-head sums over the 128 rows; the output follows one tile later
@@ -832,7 +837,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 }
 
 // One CTA per SM.  The warps of a CTA are spread over the SM's four
-// sub-partitions of 16K registers each; with 11 warps three share one, which
+// sub-partitions of 16K registers each; with 12 warps three share one, which
 // caps a thread at 168 registers.
 template <int NP, int SK, int SV, bool kFB>
 __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
@@ -861,13 +866,14 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(C::kSFull + s), 1);
+      mbar_init(bar(C::kSEmpty + s), 256);
       mbar_init(bar(C::kQFull + s), 1);
       mbar_init(bar(C::kQEmpty + s), 1);
       mbar_init(bar(C::kOFree + s), 256);
     }
     mbar_init(bar(C::kPFull), 256);
     mbar_init(bar(C::kOFull), 1);
-    mbar_init(bar(C::kDone), 1);
+    mbar_init(bar(C::kDone), 2);   // one commit from each issuing thread
     *r.abort = 0;
     *reinterpret_cast<int*>(r.smem + C::kKIssued) = 0;
     mbar_fence_init();
@@ -935,7 +941,9 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     if (warp == 0) {
       if (lane == 0) producer<NP, SK, SV, true, kFB>(a, ws, r, &tm_k, &tm_q, &tm_sk);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<NP, SK, SV, kFB>(a, ws, r);
+      if (lane == 0) s_issuer<NP, SK, SV, kFB>(a, ws, r);
+    } else if (warp == kPvWarp) {
+      if (lane == 0) pv_issuer<NP, SK, SV, kFB>(a, ws, r);
     } else if (warp == kVWarp) {
       // V loads from a warp of their own: sharing one with the K loads would
       // serialise the two threads' waits
