@@ -538,7 +538,7 @@ def extra_entries(torch, binding, world, rank, local, K):
     GQA-8, the MHA/MQA pair on identical shapes, and the paper-shaped decoder;
     then the beam step and the prefill (their own units)."""
     ex = {}
-    for name in ("gqa8_b32_m32k", "mha_b16_m16k", "mqa_b16_m16k"):
+    for name in ("gqa8_b32_m32k", "mha_b16_m16k", "mqa_b16_m16k", "long_mqa_d64_b64_m8k"):
         wl = WORKLOADS[name]
         ex[name] = decode_workload_entry(torch, binding, wl, K, resolve_path(binding, torch, "auto"), world, rank,
                                          local)

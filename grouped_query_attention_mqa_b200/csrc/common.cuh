@@ -496,7 +496,8 @@ struct DecodeArgs {
   const void* k_new;
   const void* v_new;
   const int32_t* lens;
-  int b, h, g, m_max, d;
+  int b, h, g, m_max, d;   // d: value head size d_v
+  int dk;                 // key head size d_k (q and K rows)
   int hq;
   int window;          // local attention: the newest `window` rows (0 = all rows)
   int no_merge;        // no segment spans two tiles: the decode writes every output row
@@ -533,6 +534,6 @@ cudaError_t launch_prefill_tc(void* o, const void* q, const void* k, const void*
 int tc_ctas_per_sm(int hq);
 int tc_tile_rows();
 int simt_tile_rows();
-bool tc_supported(int d, int hq);
+bool tc_supported(int d_k, int d_v, int hq);
 
 }  // namespace mqa

@@ -88,7 +88,7 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
     return MQA_ERR_INVALID_ARG;
   if ((d_k != 32 && d_k != 64 && d_k != 128) || (d_v != 32 && d_v != 64 && d_v != 128)) return MQA_ERR_UNSUPPORTED;
   const int hq = h / g;
-  const bool use_tc = dtype == MQA_BF16 && d_k == d_v && tc_supported(d_k, hq);
+  const bool use_tc = dtype == MQA_BF16 && tc_supported(d_k, d_v, hq);
   if (!use_tc && (int64_t(hq) * d_k > 4096 || int64_t(hq) * d_v > 4096)) return MQA_ERR_UNSUPPORTED;
 
   // Largest CTA count whose partials fit the array; reject when even one CTA
@@ -120,7 +120,8 @@ extern "C" mqa_status_t mqa_decode_noalloc(void* o, const void* q, const void* k
   a.h = h;
   a.g = g;
   a.m_max = m_max;
-  a.d = d_v;   // the tensor-core path has d_k == d_v
+  a.d = d_v;
+  a.dk = d_k;
   a.hq = hq;
   a.window = 0;
   a.q_beams = 0;

@@ -72,14 +72,12 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;                   // cache rows per tile (the MMA M)
-constexpr int kD = 128;                      // head size
 constexpr int kThreads = 384;                // warp 0 K/Q loads, warp 1 S products, warps 2-9 softmax, warp 10 V loads,
                                              // warp 11 P.V products
 constexpr int kVWarp = 10;
 constexpr int kPvWarp = 11;
 constexpr int kNpv = 64;                     // N of the P.V product (P padded with zero columns)
 constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte swizzle column
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
 constexpr int kSegUnits = 2;                 // cost of entering a segment, in quarter tiles (partition weight)
@@ -88,17 +86,22 @@ constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O 
 constexpr uint32_t kOCol = 128;
 constexpr uint32_t kMaxDynSmem = 232448;     // 227 KB opt-in limit per CTA
 
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, int DK, int DV>
 struct TcCfg {
   // barriers
   static constexpr int kKFull = 0, kKEmpty = SK, kVFull = 2 * SK, kVEmpty = 2 * SK + SV, kSFull = 2 * SK + 2 * SV,
                        kSEmpty = kSFull + 2, kPFull = kSEmpty + 2, kOFull = kPFull + 1, kQFull = kOFull + 1,
                        kQEmpty = kQFull + 2, kOFree = kQEmpty + 2, kDone = kOFree + 2, kNumBars = kDone + 1;
+  // head sizes: keys of DK and values of DV columns, each 64 or 128, stored as
+  // one or two 64-column halves of 128-byte swizzled rows
+  static_assert((DK == 64 || DK == 128) && (DV == 64 || DV == 128), "head sizes 64 and 128");
+  static constexpr int kKHalves = DK / 64, kVHalves = DV / 64;
+  static constexpr uint32_t kKTileBytes = kKHalves * kHalfBytes, kVTileBytes = kVHalves * kHalfBytes;
   // shared memory
   static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + SK * kTileBytes;
-  static constexpr uint32_t kQ = kV + SV * kTileBytes;
-  static constexpr uint32_t kQBytes = NP * 256;                // two 64-column halves of NP rows
+  static constexpr uint32_t kV = kK + SK * kKTileBytes;
+  static constexpr uint32_t kQ = kV + SV * kVTileBytes;
+  static constexpr uint32_t kQBytes = NP * 128 * kKHalves;    // DK/64 64-column halves of NP rows
   static constexpr uint32_t kP = kQ + 2 * kQBytes;
   static constexpr uint32_t kPBytes = kTile * 128;             // 128 rows x 64 heads (bf16)
   static constexpr uint32_t kBar = kP + kPBytes;
@@ -326,34 +329,47 @@ struct TileWalk {
 // Q of segment (seq, head) into a Q buffer (two 64-column halves of NP rows):
 // rows seq*h + head*hq.. of the 2-D map (d, b*h), or with beams the W beams'
 // q_group_heads heads of the group through the 3-D map (d, h, b*W).
+template <int DK>
 __device__ __forceinline__ void load_q(const DecodeArgs& a, const CUtensorMap* tm_q, uint32_t qdst, uint32_t bar,
                                        int seq, int head, int np) {
+  constexpr int kHalves = DK / 64;
   if (a.q_beams > 0) {
     const uint64_t pol = l2_evict_first_policy();
-    mbar_expect_tx(bar, 2u * uint32_t(a.hq) * 128u);
-    tma_load_3d(qdst, tm_q, bar, 0, head * a.q_group_heads, seq * a.q_beams, pol);
-    tma_load_3d(qdst + np * 128, tm_q, bar, 64, head * a.q_group_heads, seq * a.q_beams, pol);
+    mbar_expect_tx(bar, uint32_t(kHalves) * uint32_t(a.hq) * 128u);
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf)
+      tma_load_3d(qdst + hf * np * 128, tm_q, bar, 64 * hf, head * a.q_group_heads, seq * a.q_beams, pol);
   } else {
-    mbar_expect_tx(bar, 2u * uint32_t(np) * 128u);
+    mbar_expect_tx(bar, uint32_t(kHalves) * uint32_t(np) * 128u);
     const int qrow = seq * a.h + head * a.hq;
-    tma_load_2d(qdst, tm_q, bar, 0, qrow);
-    tma_load_2d(qdst + np * 128, tm_q, bar, 64, qrow);
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf) tma_load_2d(qdst + hf * np * 128, tm_q, bar, 64 * hf, qrow);
   }
+}
+
+// One K or V tile: W/64 boxes of 64 columns x 128 rows, one per half.
+template <int W>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int head, int row,
+                                          uint64_t pol) {
+  mbar_expect_tx(bar, uint32_t(W / 64) * kHalfBytes);
+#pragma unroll
+  for (int hf = 0; hf < W / 64; ++hf) tma_load_3d(dst + hf * kHalfBytes, map, bar, 64 * hf, head, row, pol);
 }
 
 // Fused append: write the step's new row of (sequence, K/V head) into the
 // cache at row len-1, then order that store before the tensor-memory-access
 // read of the same row.
+template <int D>
 __device__ __forceinline__ void append_new_row(const DecodeArgs& a, bool is_k, int seq, int head, int len) {
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(is_k ? a.k_new : a.v_new) +
-                                                    (int64_t(seq) * a.g + head) * kD);
+                                                    (int64_t(seq) * a.g + head) * D);
   uint4* cache = reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(
-      static_cast<const __nv_bfloat16*>(is_k ? a.k : a.v) + ((int64_t(seq) * a.m_max + (len - 1)) * a.g + head) * kD));
-  uint4 tmp[kD / 8];
+      static_cast<const __nv_bfloat16*>(is_k ? a.k : a.v) + ((int64_t(seq) * a.m_max + (len - 1)) * a.g + head) * D));
+  uint4 tmp[D / 8];
 #pragma unroll
-  for (int c = 0; c < kD / 8; ++c) tmp[c] = __ldg(src + c);
+  for (int c = 0; c < D / 8; ++c) tmp[c] = __ldg(src + c);
 #pragma unroll
-  for (int c = 0; c < kD / 8; ++c) cache[c] = tmp[c];
+  for (int c = 0; c < D / 8; ++c) cache[c] = tmp[c];
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
@@ -361,21 +377,21 @@ __device__ __forceinline__ void append_new_row(const DecodeArgs& a, bool is_k, i
 // them: Q of the segment into Q buffer 0 and the first min(2, own) K and V
 // tiles into stages 0 and 1 (K before V, as the producers order them).
 // Returns the number of tiles started; the producers skip those.
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const CUtensorMap* tm_q, const CUtensorMap* tm_sk, const CUtensorMap* tm_sv, int seq,
                          int head, int k0, int own, int len, int nb) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   static_assert(SK >= 2 && SV >= 2, "two stages of each ring");
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  load_q(a, tm_q, r.sbase + C::kQ, bar(C::kQFull), seq, head, NP);
+  load_q<DK>(a, tm_q, r.sbase + C::kQ, bar(C::kQFull), seq, head, NP);
   const int npre = own < 2 ? own : 2;
   for (int i = 0; i < npre; ++i) {
     const int k = k0 + i;
     if (a.k_new != nullptr && k == nb - 1) {
-      append_new_row(a, true, seq, head, len);
-      append_new_row(a, false, seq, head, len);
+      append_new_row<DK>(a, true, seq, head, len);
+      append_new_row<DV>(a, false, seq, head, len);
     }
     int row;
     const CUtensorMap* mk = tm_k;
@@ -392,23 +408,17 @@ __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap*
     } else {
       row = seq * a.m_max + len - span_of(len, a.window) + k * kTile;
     }
-    const uint32_t kdst = r.sbase + C::kK + i * kTileBytes;
-    mbar_expect_tx(bar(C::kKFull + i), kTileBytes);
-    tma_load_3d(kdst, mk, bar(C::kKFull + i), 0, head, row, pol);
-    tma_load_3d(kdst + kHalfBytes, mk, bar(C::kKFull + i), 64, head, row, pol);
-    const uint32_t vdst = r.sbase + C::kV + i * kTileBytes;
-    mbar_expect_tx(bar(C::kVFull + i), kTileBytes);
-    tma_load_3d(vdst, mv, bar(C::kVFull + i), 0, head, row, pol);
-    tma_load_3d(vdst + kHalfBytes, mv, bar(C::kVFull + i), 64, head, row, pol);
+    load_tile<DK>(r.sbase + C::kK + i * C::kKTileBytes, mk, bar(C::kKFull + i), head, row, pol);
+    load_tile<DV>(r.sbase + C::kV + i * C::kVTileBytes, mv, bar(C::kVFull + i), head, row, pol);
   }
   return npre;
 }
 
 // K ring and the per-segment Q (kIsK), or the V ring.
-template <int NP, int SK, int SV, bool kIsK, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kIsK, bool kFB>
 __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, const CUtensorMap* tm_kv,
                          const CUtensorMap* tm_q, const CUtensorMap* tm_skv) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   const Sched& sc = ws.s;
   constexpr int S = kIsK ? SK : SV;
   constexpr int kFull = kIsK ? C::kKFull : C::kVFull;
@@ -434,7 +444,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     if (kIsK && w.first) {
       const int qb = w.sidx & 1;
       if (w.sidx >= 2 && !wait_bar(r, bar(C::kQEmpty + qb), ((w.sidx >> 1) - 1) & 1)) break;
-      load_q(a, tm_q, r.sbase + C::kQ + qb * C::kQBytes, bar(C::kQFull + qb), w.tc.seq, w.tc.head, NP);
+      load_q<DK>(a, tm_q, r.sbase + C::kQ + qb * C::kQBytes, bar(C::kQFull + qb), w.tc.seq, w.tc.head, NP);
       q_issued = w.sidx;
     }
     const int st = int(i % S);
@@ -454,12 +464,11 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
     } else {
       row = w.tc.seq * a.m_max + w.tc.row0;
     }
-    const uint32_t dst = r.sbase + kRing + st * kTileBytes;
+    constexpr int kW = kIsK ? DK : DV;
+    const uint32_t dst = r.sbase + kRing + st * uint32_t(kW / 64) * kHalfBytes;
     if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1)   // this tile holds the sequence's newest row
-      append_new_row(a, kIsK, w.tc.seq, w.tc.head, w.len);
-    mbar_expect_tx(bar(kFull + st), kTileBytes);
-    tma_load_3d(dst, map, bar(kFull + st), 0, w.tc.head, row, pol);
-    tma_load_3d(dst + kHalfBytes, map, bar(kFull + st), 64, w.tc.head, row, pol);
+      append_new_row<kW>(a, kIsK, w.tc.seq, w.tc.head, w.len);
+    load_tile<kW>(dst, map, bar(kFull + st), w.tc.head, row, pol);
     if (kIsK) *reinterpret_cast<volatile int*>(r.smem + C::kKIssued) = int(i + 1);
   }
   // Drain: every copy this thread issued has landed before the CTA can exit.
@@ -480,9 +489,9 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
 //
 // S(j) needs K(j) landed, for a segment's first tile its Q, and S buffer j&1
 // free: the softmax warps arrive on SEmpty once they hold S(j-2) in registers.
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   const Sched& sc = ws.s;
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   const int n = int(sc.t_end - sc.t_begin);   // tiles of this CTA (fewer than 2^31)
@@ -501,11 +510,11 @@ __device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) 
     if (i >= 2 && !wait_bar(r, bar(C::kSEmpty + (i & 1)), uint32_t((i >> 1) - 1) & 1)) break;
     tc_fence_after();
     // descriptors differ only in their start address (bits 0-13, 16-byte units)
-    const uint64_t ka = kdesc0 + uint64_t((uint32_t(kst) * kTileBytes) >> 4);
+    const uint64_t ka = kdesc0 + uint64_t((uint32_t(kst) * C::kKTileBytes) >> 4);
     const uint64_t qa = qdesc0 + uint64_t((uint32_t(qb) * C::kQBytes) >> 4);
     const uint32_t d = r.tmem + uint32_t(i & 1) * NP;
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
+    for (int kk = 0; kk < DK / 16; ++kk) {
       const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
       const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
       mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
@@ -525,14 +534,17 @@ __device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) 
 
 // O += V^T P(j) needs P(j) written, V(j) landed and, for a segment's first
 // tile, its O buffer released by the epilogue of the segment two back.
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   const Sched& sc = ws.s;
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int n = int(sc.t_end - sc.t_begin);
   TileWalk<kFB> w(a, ws, r);
-  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, kHalfBytes, 1024);   // MN-major V^T
+  // MN-major V^T; its M (V columns) is always 128: with DV = 64 the second
+  // 64-column atom points back at the first (leading offset 0), and the
+  // duplicated half of O is never written out.
+  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, DV == 128 ? kHalfBytes : 0u, 1024);
   const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);   // MN-major P
   const uint32_t bar0 = r.sbase + C::kBar;
   auto bar = [&](int id) { return bar0 + 8u * uint32_t(id); };
@@ -545,7 +557,7 @@ __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r)
     if (!wait_bar(r, bar(C::kVFull + vst), vph)) break;
     if (w.first && w.sidx >= 2 && !wait_bar(r, bar(C::kOFree + ob), uint32_t((w.sidx >> 1) - 1) & 1)) break;
     tc_fence_after();
-    const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * kTileBytes) >> 4);
+    const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * C::kVTileBytes) >> 4);
     const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
     const uint32_t acc0 = w.first ? 0u : 1u;
 #pragma unroll
@@ -562,9 +574,9 @@ __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r)
   mbar_wait(bar(C::kDone), 0, kTimeoutNs);
 }
 
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Roles& r, int warp, int lane) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   const Sched& sc = ws.s;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   auto wait = [&](int id, uint32_t parity) { return mbar_wait(bar(id), parity, kTimeoutNs); };
@@ -618,7 +630,9 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     const int64_t slot = partial_slot(blockIdx.x, e.seg);
     float v[CPT];
     tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
-    if (e.whole) {
+    if (row >= DV) {
+      // columns past DV only repeat the first ones (see the P.V descriptor)
+    } else if (e.whole) {
       if constexpr (kFB) {   // column (w, i) of the segment is head i of the group in beam w's output row
         const int qgh = a.q_group_heads;
         int bw = col0 / qgh, bi = col0 - bw * qgh;
@@ -626,7 +640,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
         for (int k = 0; k < CPT; ++k) {
           if (col0 + k < hq)
             static_cast<__nv_bfloat16*>(a.o)[((int64_t(e.seq) * a.q_beams + bw) * a.h + int64_t(e.head) * qgh + bi) *
-                                                 kD + row] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+                                                 DV + row] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
           if (++bi == qgh) {
             bi = 0;
             ++bw;
@@ -634,16 +648,16 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
         }
       } else {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) +
-                             (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * kD + row;
+                             (int64_t(e.seq) * a.h + int64_t(e.head) * hq + col0) * DV + row;
 #pragma unroll
         for (int k = 0; k < CPT; ++k)
-          if (col0 + k < hq) dst[k * kD] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
+          if (col0 + k < hq) dst[k * DV] = __float2bfloat16_rn(v[k] * linv[pb * NP + col0 + k]);
       }
     } else {
-      float* dst = a.ws.part_o + (slot * hq + col0) * kD + row;
+      float* dst = a.ws.part_o + (slot * hq + col0) * DV + row;
 #pragma unroll
       for (int k = 0; k < CPT; ++k)
-        if (col0 + k < hq) dst[k * kD] = v[k] * linv[pb * NP + col0 + k];
+        if (col0 + k < hq) dst[k * DV] = v[k] * linv[pb * NP + col0 + k];
     }
     if (warp == 2) {
       if (!e.whole)   // every partial carries its log-sum-exp
@@ -773,10 +787,10 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       // rows past the sequence end were loaded too; zero them in V so that
       // P = 0 times whatever they hold contributes exactly 0.  Consecutive
       // threads take consecutive 16-byte pieces of a row (no bank conflicts).
-      unsigned char* vst = r.smem + C::kV + st * kTileBytes;
-      const int nchunks = (kTile - w.tc.rows) * 16;
+      unsigned char* vst = r.smem + C::kV + st * C::kVTileBytes;
+      const int nchunks = (kTile - w.tc.rows) * 8 * C::kVHalves;
       for (int k = tid; k < nchunks; k += 256) {
-        const int vr = w.tc.rows + (k >> 4), half = (k >> 3) & 1, c16 = k & 7;
+        const int vr = w.tc.rows + k / (8 * C::kVHalves), half = (k >> 3) & (C::kVHalves - 1), c16 = k & 7;
         *reinterpret_cast<uint4*>(vst + half * kHalfBytes + (vr >> 3) * 1024 + (vr & 7) * 128 + c16 * 16) =
             make_uint4(0, 0, 0, 0);
       }
@@ -839,11 +853,11 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 // One CTA per SM.  The warps of a CTA are spread over the SM's four
 // sub-partitions of 16K registers each; with 12 warps three share one, which
 // caps a thread at 168 registers.
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                                const CUtensorMap& tm_q, const CUtensorMap& tm_sk,
                                                const CUtensorMap& tm_sv) {
-  using C = TcCfg<NP, SK, SV>;
+  using C = TcCfg<NP, SK, SV, DK, DV>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -913,7 +927,7 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
         a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
         kFB ? reinterpret_cast<int*>(r.smem + C::kNsuf) : nullptr,
         [&](int seq, int head, int k0, int own, int len, int nb) {
-          return pre_issue<NP, SK, SV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, k0, own, len, nb);
+          return pre_issue<NP, SK, SV, DK, DV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, k0, own, len, nb);
         });
     r.seq0 = 0;
     if (kFB) r.nsuf_s = reinterpret_cast<const int*>(r.smem + C::kNsuf);
@@ -931,25 +945,25 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
   if (a.no_merge && warp >= 2 && warp < kVWarp) {   // no merge follows: empty sequences get their zero rows here
     for (int s = blockIdx.x; s < a.b; s += gridDim.x) {
       if (clamp_len(__ldg(a.lens + s), a.m_max, nullptr, false) == 0) {
-        uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + int64_t(s) * a.h * kD);
-        for (int k = int(threadIdx.x) - 64; k < a.h * kD / 8; k += 256) o[k] = make_uint4(0, 0, 0, 0);
+        uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + int64_t(s) * a.h * DV);
+        for (int k = int(threadIdx.x) - 64; k < a.h * DV / 8; k += 256) o[k] = make_uint4(0, 0, 0, 0);
       }
     }
   }
 
   if (sc.t_begin < sc.t_end) {
     if (warp == 0) {
-      if (lane == 0) producer<NP, SK, SV, true, kFB>(a, ws, r, &tm_k, &tm_q, &tm_sk);
+      if (lane == 0) producer<NP, SK, SV, DK, DV, true, kFB>(a, ws, r, &tm_k, &tm_q, &tm_sk);
     } else if (warp == 1) {
-      if (lane == 0) s_issuer<NP, SK, SV, kFB>(a, ws, r);
+      if (lane == 0) s_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
     } else if (warp == kPvWarp) {
-      if (lane == 0) pv_issuer<NP, SK, SV, kFB>(a, ws, r);
+      if (lane == 0) pv_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
     } else if (warp == kVWarp) {
       // V loads from a warp of their own: sharing one with the K loads would
       // serialise the two threads' waits
-      if (lane == 0) producer<NP, SK, SV, false, kFB>(a, ws, r, &tm_v, &tm_q, &tm_sv);
+      if (lane == 0) producer<NP, SK, SV, DK, DV, false, kFB>(a, ws, r, &tm_v, &tm_q, &tm_sv);
     } else {
-      softmax_epilogue<NP, SK, SV, kFB>(a, ws, r, warp, lane);
+      softmax_epilogue<NP, SK, SV, DK, DV, kFB>(a, ws, r, warp, lane);
     }
   }
   tc_fence_before();
@@ -961,20 +975,20 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
   asm volatile("griddepcontrol.launch_dependents;");
 }
 
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
-  decode_tc_body<NP, SK, SV, false>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
+  decode_tc_body<NP, SK, SV, DK, DV, false>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
 }
 
 // Beams sharing a prefix in one pass: the suffix caches' maps as well.
-template <int NP, int SK, int SV>
+template <int NP, int SK, int SV, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_beam_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_sk, const __grid_constant__ CUtensorMap tm_sv) {
-  decode_tc_body<NP, SK, SV, true>(a, tm_k, tm_v, tm_q, tm_sk, tm_sv);
+  decode_tc_body<NP, SK, SV, DK, DV, true>(a, tm_k, tm_v, tm_q, tm_sk, tm_sv);
 }
 
 // ------------------------------------------------------------------ host
@@ -995,11 +1009,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Cache [b, m_max, g, 128] bf16 as a 3-D tensor (d, g, b*m_max); a box is 64
-// columns of one K/V head over 128 consecutive rows, 128-byte swizzled.
-bool encode_cache(CUtensorMap* m, const void* base, int b, int m_max, int g) {
-  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(g), cuuint64_t(b) * cuuint64_t(m_max)};
-  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(g) * kD * 2};
+// Cache [b, m_max, g, d] bf16 (d = 64 or 128) as a 3-D tensor (d, g, b*m_max);
+// a box is 64 columns of one K/V head over 128 consecutive rows, 128-byte
+// swizzled.
+bool encode_cache(CUtensorMap* m, const void* base, int b, int m_max, int g, int d) {
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(g), cuuint64_t(b) * cuuint64_t(m_max)};
+  const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(g) * cuuint64_t(d) * 2};
   const cuuint32_t box[3] = {64, 1, kTile};
   const cuuint32_t estr[3] = {1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -1007,11 +1022,11 @@ bool encode_cache(CUtensorMap* m, const void* base, int b, int m_max, int g) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// q [b*h, 128] bf16; a box is 64 columns of NP consecutive heads.
+// q [b*h, d_k] bf16; a box is 64 columns of NP consecutive heads.
 // Beam queries [b*W, h, d] as (d, h, b*W) with boxes of 64 x heads x W.
-bool encode_q_beams(CUtensorMap* m, const void* base, int h, int rows, int heads, int beams) {
-  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h), cuuint64_t(rows)};
-  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(h) * kD * 2};
+bool encode_q_beams(CUtensorMap* m, const void* base, int h, int rows, int heads, int beams, int d) {
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(h), cuuint64_t(rows)};
+  const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(h) * cuuint64_t(d) * 2};
   const cuuint32_t box[3] = {64, cuuint32_t(heads), cuuint32_t(beams)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -1019,9 +1034,9 @@ bool encode_q_beams(CUtensorMap* m, const void* base, int h, int rows, int heads
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_q(CUtensorMap* m, const void* base, int rows, int np) {
-  const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kD) * 2};
+bool encode_q(CUtensorMap* m, const void* base, int rows, int np, int d) {
+  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
   const cuuint32_t box[2] = {64, cuuint32_t(np)};
   const cuuint32_t estr[2] = {1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -1029,29 +1044,29 @@ bool encode_q(CUtensorMap* m, const void* base, int rows, int np) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NP, int SK, int SV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
-  using L = TcCfg<NP, SK, SV>;
+  using L = TcCfg<NP, SK, SV, DK, DV>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = kFB ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = kFB ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    int(L::kAlloc))
-            : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    int(L::kAlloc));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tk, tv, tq, tsk, tsv;
-  if (!encode_cache(&tk, a.k, a.b, a.m_max, a.g) || !encode_cache(&tv, a.v, a.b, a.m_max, a.g) ||
-      !(a.q_beams > 0 ? encode_q_beams(&tq, a.q, a.h, a.b * a.q_beams, a.q_group_heads, a.q_beams)
-                      : encode_q(&tq, a.q, a.b * a.h, NP)))
+  if (!encode_cache(&tk, a.k, a.b, a.m_max, a.g, DK) || !encode_cache(&tv, a.v, a.b, a.m_max, a.g, DV) ||
+      !(a.q_beams > 0 ? encode_q_beams(&tq, a.q, a.h, a.b * a.q_beams, a.q_group_heads, a.q_beams, DK)
+                      : encode_q(&tq, a.q, a.b * a.h, NP, DK)))
     return cudaErrorInvalidValue;
-  if (kFB && (!encode_cache(&tsk, a.sk, a.b * a.q_beams, a.m_s, a.g) ||
-              !encode_cache(&tsv, a.sv, a.b * a.q_beams, a.m_s, a.g)))
+  if (kFB && (!encode_cache(&tsk, a.sk, a.b * a.q_beams, a.m_s, a.g, DK) ||
+              !encode_cache(&tsv, a.sv, a.b * a.q_beams, a.m_s, a.g, DV)))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(a.grid));
@@ -1063,13 +1078,23 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV>, a, tk, tv, tq, tsk, tsv);
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NP, SK, SV>, a, tk, tv, tq);
+  if (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq, tsk, tsv);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq);
+}
+
+template <int SK, int SV, int DK, int DV>
+cudaError_t launch_hq(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.hq <= 16) return launch_np<16, SK, SV, DK, DV, false>(a, stream);
+  if (a.hq <= 32) return launch_np<32, SK, SV, DK, DV, false>(a, stream);
+  if (a.hq <= 64) return launch_np<64, SK, SV, DK, DV, false>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool tc_supported(int d, int hq) { return d == kD && hq >= 1 && hq <= 64; }
+bool tc_supported(int d_k, int d_v, int hq) {
+  return (d_k == 64 || d_k == 128) && (d_v == 64 || d_v == 128) && hq >= 1 && hq <= 64;
+}
 
 int tc_ctas_per_sm(int) { return 1; }
 
@@ -1078,16 +1103,19 @@ int tc_tile_rows() { return kTile; }
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) || int64_t(a.b) * a.h >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
-  if (a.sk != nullptr) {   // beams sharing a prefix, one pass
+  if (a.sk != nullptr) {   // beams sharing a prefix, one pass (head size 128)
     if (a.q_beams < 1 || int64_t(a.b) * a.q_beams * a.m_s >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-    if (a.hq <= 16) return launch_np<16, 2, 3, true>(a, stream);
-    if (a.hq <= 32) return launch_np<32, 2, 3, true>(a, stream);
-    if (a.hq <= 64) return launch_np<64, 2, 3, true>(a, stream);
+    if (a.dk != 128 || a.d != 128) return cudaErrorInvalidValue;
+    if (a.hq <= 16) return launch_np<16, 2, 3, 128, 128, true>(a, stream);
+    if (a.hq <= 32) return launch_np<32, 2, 3, 128, 128, true>(a, stream);
+    if (a.hq <= 64) return launch_np<64, 2, 3, 128, 128, true>(a, stream);
     return cudaErrorInvalidValue;
   }
-  if (a.hq <= 16) return launch_np<16, 2, 3, false>(a, stream);
-  if (a.hq <= 32) return launch_np<32, 2, 3, false>(a, stream);
-  if (a.hq <= 64) return launch_np<64, 2, 3, false>(a, stream);
+  // Ring stages: about 64 KB of K and 96 KB of V tiles whatever the head sizes.
+  if (a.dk == 128 && a.d == 128) return launch_hq<2, 3, 128, 128>(a, stream);
+  if (a.dk == 64 && a.d == 64) return launch_hq<4, 6, 64, 64>(a, stream);
+  if (a.dk == 128 && a.d == 64) return launch_hq<2, 6, 128, 64>(a, stream);
+  if (a.dk == 64 && a.d == 128) return launch_hq<4, 3, 64, 128>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -90,7 +90,7 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   if (workspace_bytes_given < workspace_bytes(b, g, hq, d_v)) return MQA_ERR_INVALID_ARG;
   if ((d_k != 32 && d_k != 64 && d_k != 128) || (d_v != 32 && d_v != 64 && d_v != 128)) return MQA_ERR_UNSUPPORTED;
 
-  const bool tc_ok = dtype == MQA_BF16 && d_k == d_v && tc_supported(d_k, hq);
+  const bool tc_ok = dtype == MQA_BF16 && tc_supported(d_k, d_v, hq);
   const bool simt_ok = int64_t(hq) * d_k <= 4096 && int64_t(hq) * d_v <= 4096;
   bool use_tc;
   if (path == MQA_PATH_TCGEN05) {
@@ -118,7 +118,8 @@ mqa_status_t decode_impl(void* o, const void* q, const void* k_cache, const void
   a.h = h;
   a.g = g;
   a.m_max = m_max;
-  a.d = d_v;   // the tensor-core path has d_k == d_v
+  a.d = d_v;
+  a.dk = d_k;
   a.hq = hq;
   a.window = opts ? opts->window : 0;
   a.q_beams = 0;
@@ -181,7 +182,7 @@ mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const
     return MQA_ERR_INVALID_ARG;
   const int hq = h / g;
   if (workspace_bytes_given < mqa_decode_beam_workspace_size(b, W, h, g, d_v)) return MQA_ERR_INVALID_ARG;
-  if (dtype != MQA_BF16 || d_k != d_v || !tc_supported(d_k, W * hq)) return MQA_ERR_UNSUPPORTED;
+  if (dtype != MQA_BF16 || d_k != 128 || d_v != 128 || !tc_supported(d_k, d_v, W * hq)) return MQA_ERR_UNSUPPORTED;
   const int sms = sm_count();
   if (sms <= 0) return MQA_ERR_CUDA;
   // One pass: segment (s, j) reads sequence s's prefix once for the W beams'
@@ -199,7 +200,8 @@ mqa_status_t mqa_decode_beam(void* o, const void* q, const void* prefix_k, const
   a.h = h;
   a.g = g;
   a.m_max = m_p;
-  a.d = d_k;
+  a.d = d_v;
+  a.dk = d_k;
   a.hq = W * hq;
   a.window = 0;
   a.no_merge = 0;

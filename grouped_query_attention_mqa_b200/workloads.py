@@ -101,6 +101,10 @@ WORKLOADS = {
         "long_mqa_b64_m8k", b=64, h=32, g=1, d_k=128, d_v=128, m_max=8192, len_lo=1024, len_hi=8192,
         dtype="bf16", scale=1.0, q_std=_S128,
         description="long-context MQA serving batch: b=64 h=32 g=1 d=128 m_max=8192, lens U[1024,8192]"),
+    "long_mqa_d64_b64_m8k": Workload(
+        "long_mqa_d64_b64_m8k", b=64, h=32, g=1, d_k=64, d_v=64, m_max=8192, len_lo=1024, len_hi=8192,
+        dtype="bf16", scale=1.0, q_std=1.0 / math.sqrt(64.0),
+        description="long-context MQA batch with head size 64: b=64 h=32 g=1 d=64 m_max=8192, lens U[1024,8192]"),
     "gqa8_b32_m32k": Workload(
         "gqa8_b32_m32k", b=32, h=64, g=8, d_k=128, d_v=128, m_max=32768, len_lo=8192, len_hi=32768,
         dtype="bf16", scale=_S128,

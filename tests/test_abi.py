@@ -85,8 +85,9 @@ def test_decode_rejects_bad_arguments_without_launching(lib):
     assert _decode(lib, m_max=0) == INV
     assert _decode(lib, d_k=96, d_v=96) == UNS           # head size not built
     assert _decode(lib, d_k=128, d_v=96) == UNS          # value width not built
-    opts = binding.DecodeOptions(2, 0)                   # tensor cores: d_k = d_v only
-    assert _decode(lib, d_k=128, d_v=64, opts=ctypes.byref(opts)) == UNS
+    opts = binding.DecodeOptions(2, 0)                   # tensor cores: head sizes 64 and 128 only
+    assert _decode(lib, d_k=128, d_v=32, opts=ctypes.byref(opts)) == UNS
+    assert _decode(lib, d_k=32, d_v=64, opts=ctypes.byref(opts)) == UNS
     opts = binding.DecodeOptions(1, 0)                   # SIMT: h/g * d_v <= 4096 as well
     assert _decode(lib, h=64, d_k=32, d_v=128, opts=ctypes.byref(opts)) == UNS
     opts = binding.DecodeOptions(9, 0)
@@ -144,8 +145,8 @@ def test_fused_step_rejects_bad_arguments_without_launching(lib):
     assert _fused(lib, g=3) == INV
     assert _fused(lib, ws_bytes=100) == INV
     assert _fused(lib, d_k=96, d_v=96) == UNS
-    opts = binding.DecodeOptions(2, 0)                   # tensor cores: d_k = d_v only
-    assert _fused(lib, d_v=64, opts=ctypes.byref(opts)) == UNS
+    opts = binding.DecodeOptions(2, 0)                   # tensor cores: head sizes 64 and 128 only
+    assert _fused(lib, d_v=32, opts=ctypes.byref(opts)) == UNS
     assert _fused(lib, b=0, kn=None, vn=None) == binding.MQA_OK
 
 

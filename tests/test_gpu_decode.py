@@ -25,7 +25,8 @@ def _lib():
 
 
 def tc_available(wl):
-    return wl.dtype == "bf16" and wl.d_k == 128 and 1 <= wl.heads_per_group <= 64 and _tc_built()
+    return (wl.dtype == "bf16" and wl.d_k in (64, 128) and wl.d_v in (64, 128) and 1 <= wl.heads_per_group <= 64
+            and _tc_built())
 
 
 def _tc_built():

@@ -1,11 +1,12 @@
-"""Keys and values of different widths (d_k != d_v) on the CUDA-core decode.
+"""Keys and values of different widths (d_k != d_v).
 
 The paper's per-head sizes are k for queries and keys and v for values and
 outputs, and nothing in the method ties them together ("Fast Transformer
 Decoding", velog paper review §2.4 and §3: logits over the k axis, outputs
 over the v axis).  Every pairing of d_k, d_v in {32, 64, 128} is built on the
-CUDA-core path; the tensor-core path keeps d_k = d_v = 128 and the automatic
-choice falls back to the CUDA-core path for unequal widths.  Compared element
+CUDA-core path; the tensor-core path takes bf16 pairings of 64 and 128, and
+the automatic choice takes it there.  Each bf16 case runs on the automatic
+choice and on the CUDA-core path.  Compared element
 by element with the float64 oracle on seeded inputs whose masked rows hold
 NaN, with sequences split between CTAs (merge) and kept whole, through the
 fused append + decode step (cache bits checked exactly), the local window and
@@ -50,13 +51,16 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["auto", "simt"])
 @pytest.mark.parametrize("num_ctas", [0, 1, 5])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "_".join(map(str, s[:7])))
-def test_unequal_widths_match_oracle(shape, num_ctas):
+def test_unequal_widths_match_oracle(shape, num_ctas, path):
     wl = wl_of(*shape)
+    if path == "simt" and wl.dtype == "f32":
+        pytest.skip("fp32 always takes the CUDA-core path")
     inp = host_inputs(wl, seed=7 + num_ctas, nan_tail=True)
     o = binding.decode(dev(inp["q"], wl.dtype), dev(inp["k"], wl.dtype), dev(inp["v"], wl.dtype),
-                       torch.from_numpy(inp["lens"]).cuda(), wl.scale, num_ctas=num_ctas)
+                       torch.from_numpy(inp["lens"]).cuda(), wl.scale, num_ctas=num_ctas, path=path)
     torch.cuda.synchronize()
     assert tuple(o.shape) == (wl.b, wl.h, wl.d_v)
     ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], inp["lens"], wl.g, wl.scale)
@@ -114,8 +118,10 @@ def test_window_unequal_widths():
         assert_close(host64(o), ref, "bf16", f"window={window}")
 
 
-def test_tensor_core_path_keeps_equal_widths():
-    wl = wl_of("bf16", 1, 8, 1, 128, 64, 16, 1, 16)
+def test_tensor_core_path_takes_head_sizes_64_and_128_only():
+    """Keys and values of 64 or 128 columns, in any pairing, are served by the
+    tensor-core path; a 32-column head is not (it stays on the CUDA cores)."""
+    wl = wl_of("bf16", 1, 8, 1, 32, 128, 16, 1, 16)
     inp = host_inputs(wl, seed=1)
     with pytest.raises(binding.MqaError) as e:
         binding.decode(dev(inp["q"], "bf16"), dev(inp["k"], "bf16"), dev(inp["v"], "bf16"),
