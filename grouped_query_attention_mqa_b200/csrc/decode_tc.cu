@@ -22,7 +22,7 @@
 //
 // Work: one CTA per SM, persistent over a contiguous run of all segments'
 // tiles; runs are balanced in quarter tiles with a segment's entry weighted
-// as half a tile.  The thread of the schedule that finds a CTA's first tile
+// as a whole tile.  The thread of the schedule that finds a CTA's first tile
 // issues its first Q, K and V loads itself (start-up code runs at
 // instruction-fetch speed; a separate role would reach them much later).
 // A segment split between CTAs leaves normalised partials with their
@@ -80,7 +80,7 @@ constexpr int kNpv = 64;                     // N of the P.V product (P padded w
 constexpr uint32_t kHalfBytes = kTile * 128; // 128 rows x 64 bf16, one 128-byte swizzle column
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
-constexpr int kSegUnits = 2;                 // cost of entering a segment, in quarter tiles (partition weight)
+constexpr int kSegUnits = 4;                 // cost of entering a segment, in quarter tiles (partition weight)
 constexpr int kLensCache = kThreads;         // clamped lengths kept in shared memory (all of them when b <= kThreads)
 constexpr uint32_t kTmemCols = 256;          // S double buffer at [0, 2*NP), O double buffer at [128, 256)
 constexpr uint32_t kOCol = 128;
