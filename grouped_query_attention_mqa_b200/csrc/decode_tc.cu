@@ -574,6 +574,101 @@ __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r)
   mbar_wait(bar(C::kDone), 0, kTimeoutNs);
 }
 
+// The beam kernel keeps one thread for both streams: S(j) = K Q^T once K(j)
+// (and a segment's Q) has landed and P(j-2) has been consumed (j <= i + 1),
+// O += V^T P(i) once P(i) and V(i) are there; it polls both and issues
+// whichever is ready, with ring stages and phase parities advanced by
+// increments.  (Its walker reads the suffix lengths of every beam; a copy per
+// stream measured slower than one thread serving both.)
+template <int NP, int SK, int SV, int DK, int DV, bool kFB>
+__device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
+  using C = TcCfg<NP, SK, SV, DK, DV>;
+  const Sched& sc = ws.s;
+  constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
+  const int n = int(sc.t_end - sc.t_begin);
+  TileWalk<kFB> wq(a, ws, r), wp(a, ws, r);
+  const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);
+  const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
+  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, DV == 128 ? kHalfBytes : 0u, 1024);
+  const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);
+  const uint32_t bar0 = r.sbase + C::kBar;
+  auto bar = [&](int id) { return bar0 + 8u * uint32_t(id); };
+  int iq = 0, ip = 0, kst = 0, vst = 0;
+  uint32_t kph = 0, vph = 0;
+  if (n > 0) {
+    wq.next(a, sc);
+    wp.next(a, sc);
+  }
+  uint64_t idle_since = 0;
+  uint32_t idle_polls = 0;
+  while (ip < n) {
+    bool progressed = false;
+    if (iq < n && iq <= ip + 1) {
+      const int qb = wq.sidx & 1;
+      if ((!wq.first || mbar_test(bar(C::kQFull + qb), uint32_t(wq.sidx >> 1) & 1)) &&
+          mbar_test(bar(C::kKFull + kst), kph)) {
+        tc_fence_after();
+        const uint64_t ka = kdesc0 + uint64_t((uint32_t(kst) * C::kKTileBytes) >> 4);
+        const uint64_t qa = qdesc0 + uint64_t((uint32_t(qb) * C::kQBytes) >> 4);
+        const uint32_t d = r.tmem + uint32_t(iq & 1) * NP;
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
+        }
+        mma_commit(bar(C::kSFull + (iq & 1)));
+        mma_commit(bar(C::kKEmpty + kst));
+        if (wq.last) mma_commit(bar(C::kQEmpty + qb));
+        ++iq;
+        if (++kst == SK) {
+          kst = 0;
+          kph ^= 1u;
+        }
+        if (iq < n) wq.next(a, sc);
+        progressed = true;
+      }
+    }
+    if (ip < iq) {
+      const int ob = wp.sidx & 1;
+      if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) && mbar_test(bar(C::kVFull + vst), vph) &&
+          (!wp.first || wp.sidx < 2 || mbar_test(bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))) {
+        tc_fence_after();
+        const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * C::kVTileBytes) >> 4);
+        const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
+        const uint32_t acc0 = wp.first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        mma_commit(bar(C::kOFull));
+        mma_commit(bar(C::kVEmpty + vst));
+        ++ip;
+        if (++vst == SV) {
+          vst = 0;
+          vph ^= 1u;
+        }
+        if (ip < n) wp.next(a, sc);
+        progressed = true;
+      }
+    }
+    if (progressed) {
+      idle_polls = 0;
+    } else if ((++idle_polls & 1023u) == 0) {   // bounded: give up after the timeout without progress
+      const uint64_t now = globaltimer_ns();
+      if (idle_polls == 1024) {
+        idle_since = now;
+      } else if (now - idle_since > kTimeoutNs || *r.abort) {
+        *r.abort = 1;
+        set_flag(r.flags, MQA_FLAG_PIPE_TIMEOUT);
+        break;
+      }
+    }
+  }
+  mma_commit(bar(C::kDone));
+  mbar_wait(bar(C::kDone), 0, kTimeoutNs);
+}
+
 template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Roles& r, int warp, int lane) {
   using C = TcCfg<NP, SK, SV, DK, DV>;
@@ -887,7 +982,7 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     }
     mbar_init(bar(C::kPFull), 256);
     mbar_init(bar(C::kOFull), 1);
-    mbar_init(bar(C::kDone), 2);   // one commit from each issuing thread
+    mbar_init(bar(C::kDone), kFB ? 1 : 2);   // one commit from each issuing thread
     *r.abort = 0;
     *reinterpret_cast<int*>(r.smem + C::kKIssued) = 0;
     mbar_fence_init();
@@ -955,9 +1050,12 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     if (warp == 0) {
       if (lane == 0) producer<NP, SK, SV, DK, DV, true, kFB>(a, ws, r, &tm_k, &tm_q, &tm_sk);
     } else if (warp == 1) {
-      if (lane == 0) s_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
+      if (lane == 0) {
+        if constexpr (kFB) mma_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
+        else s_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
+      }
     } else if (warp == kPvWarp) {
-      if (lane == 0) pv_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
+      if (!kFB && lane == 0) pv_issuer<NP, SK, SV, DK, DV, kFB>(a, ws, r);
     } else if (warp == kVWarp) {
       // V loads from a warp of their own: sharing one with the K loads would
       // serialise the two threads' waits
