@@ -948,7 +948,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 // One CTA per SM.  The warps of a CTA are spread over the SM's four
 // sub-partitions of 16K registers each; with 12 warps three share one, which
 // caps a thread at 168 registers.
-template <int NP, int SK, int SV, int DK, int DV, bool kFB>
+template <int NP, int SK, int SV, int DK, int DV, bool kFB, bool kOne>
 __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                                const CUtensorMap& tm_q, const CUtensorMap& tm_sk,
                                                const CUtensorMap& tm_sv) {
@@ -1016,8 +1016,34 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     bs.W = 0;
     bs.m_s = 0;
   }
-  if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
-                          kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
+  if constexpr (kOne) {
+    // Every attended span fits one tile and there are no more (sequence,
+    // K/V head) segments than CTAs: CTA c takes segment c whole, its only
+    // tile.  No scan: one length load, then at once the loads of the
+    // segment's Q, K and V.
+    const int c = blockIdx.x, nseg = a.b * a.g;
+    const int seq = c < nseg ? c / a.g : 0, head = c < nseg ? c - seq * a.g : 0;
+    if (threadIdx.x == 0) {
+      const int len = c < nseg ? clamp_len(__ldg(a.lens + seq), a.m_max, a.flags, head == 0) : 0;
+      lens_tab[0] = len;
+      sched_red[0] = len > 0 ? pre_issue<NP, SK, SV, DK, DV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head,
+                                                                 0, 1, len, 1)
+                             : 0;
+    }
+    __syncthreads();
+    const bool work = lens_tab[0] > 0;
+    ws.s.total = nseg;
+    ws.s.active = a.grid;
+    ws.s.t_begin = work ? c : 0;   // numbered per sequence: segment (seq, head) is tile seq*g + head
+    ws.s.t_end = work ? c + 1 : 0;
+    ws.s.seq = seq;
+    ws.s.seq_base = int64_t(seq) * a.g;
+    ws.wtotal = 1;
+    ws.seq_ubase = 0;
+    ws.pre = int(sched_red[0]);
+    r.seq0 = seq;   // lens_tab[0] holds this sequence's length
+  } else if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
+                                 kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
     ws = make_schedule_small<kThreads>(
         a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
         kFB ? reinterpret_cast<int*>(r.smem + C::kNsuf) : nullptr,
@@ -1077,7 +1103,16 @@ template <int NP, int SK, int SV, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
-  decode_tc_body<NP, SK, SV, DK, DV, false>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
+  decode_tc_body<NP, SK, SV, DK, DV, false, false>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
+}
+
+// Single-tile spans with no more segments than CTAs: one segment per CTA.  A
+// kernel of its own, so that the general kernel carries none of its code.
+template <int NP, int SK, int SV, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_one_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
+  decode_tc_body<NP, SK, SV, DK, DV, false, true>(a, tm_k, tm_v, tm_q, tm_k, tm_v);
 }
 
 // Beams sharing a prefix in one pass: the suffix caches' maps as well.
@@ -1086,7 +1121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_beam_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_sk, const __grid_constant__ CUtensorMap tm_sv) {
-  decode_tc_body<NP, SK, SV, DK, DV, true>(a, tm_k, tm_v, tm_q, tm_sk, tm_sv);
+  decode_tc_body<NP, SK, SV, DK, DV, true, false>(a, tm_k, tm_v, tm_q, tm_sk, tm_sv);
 }
 
 // ------------------------------------------------------------------ host
@@ -1145,17 +1180,20 @@ bool encode_q(CUtensorMap* m, const void* base, int rows, int np, int d) {
 template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   using L = TcCfg<NP, SK, SV, DK, DV>;
-  static bool attr_set[64] = {false};
+  const bool one = !kFB && a.no_merge && int64_t(a.b) * a.g <= a.grid;
+  static bool attr_set[2][64] = {{false}};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = kFB ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(L::kAlloc))
-            : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(L::kAlloc));
+  if (dev < 0 || dev >= 64 || !attr_set[one][dev]) {
+    e = kFB  ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc))
+        : one ? cudaFuncSetAttribute(decode_tc_one_kernel<NP, SK, SV, DK, DV>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc))
+              : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV, DK, DV>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc));
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[one][dev] = true;
   }
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tk, tv, tq, tsk, tsv;
@@ -1177,6 +1215,12 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq, tsk, tsv);
+  if (one) {   // one CTA per segment, none idle
+    DecodeArgs a1 = a;
+    a1.grid = a.b * a.g;
+    cfg.gridDim = dim3(unsigned(a1.grid));
+    return cudaLaunchKernelEx(&cfg, decode_tc_one_kernel<NP, SK, SV, DK, DV>, a1, tk, tv, tq);
+  }
   return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq);
 }
 
