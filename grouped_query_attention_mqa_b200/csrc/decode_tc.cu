@@ -96,7 +96,19 @@ struct TcCfg {
   // one or two 64-column halves of 128-byte swizzled rows
   static_assert((DK == 64 || DK == 128) && (DV == 64 || DV == 128), "head sizes 64 and 128");
   static constexpr int kKHalves = DK / 64, kVHalves = DV / 64;
-  static constexpr uint32_t kKTileBytes = kKHalves * kHalfBytes, kVTileBytes = kVHalves * kHalfBytes;
+  // Head size 64 with at most 32 heads per group: a tile is 256 rows, two
+  // 128-row halves.  Both halves' S products land side by side in tensor
+  // memory (the second at column kNpv/2), their P rows share the P buffer's
+  // lines, and one P.V product takes V's two row halves as the two 64-row
+  // halves of its M = 128, so a 256-row tile costs the MMAs of a 128-row tile
+  // at head size 128.  The second half's output is in lanes 64-127 at columns
+  // kNpv/2 + head and is added to the first's in the epilogue.
+  static constexpr bool kPair = DK == 64 && DV == 64 && NP <= kNpv / 2;
+  static constexpr int kRowHalves = kPair ? 2 : 1;
+  static constexpr int kRows = kRowHalves * kTile;             // cache rows per tile
+  static constexpr uint32_t kSStride = kPair ? kNpv : NP;      // tensor-memory columns per S buffer
+  static constexpr uint32_t kKTileBytes = kRowHalves * kKHalves * kHalfBytes,
+                            kVTileBytes = kRowHalves * kVHalves * kHalfBytes;
   // shared memory
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + SK * kKTileBytes;
@@ -118,7 +130,8 @@ struct TcCfg {
   static constexpr uint32_t kKIssued = kLens + kLensCache * 4;   // K tiles issued so far (V producer trails it)
   static constexpr uint32_t kSched = kKIssued + 16;            // start-up scratch of the schedule
   static constexpr uint32_t kNsuf = kSched + 256;              // [kLensCache] beams: suffix tiles per sequence
-  static constexpr uint32_t kEnd = kNsuf + kLensCache * 4;
+  static constexpr uint32_t kX = kNsuf + kLensCache * 4;       // [NP][64] f32: second row half's output
+  static constexpr uint32_t kEnd = kX + (kPair ? NP * 64 * 4 : 0);
   static constexpr uint32_t kAlloc = kEnd + 1024;             // room to align the base to 1024 bytes
   static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kQBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
   static_assert(kAlloc <= kMaxDynSmem, "shared memory budget");
@@ -254,7 +267,7 @@ __device__ __forceinline__ void locate_tile(const DecodeArgs& a, int seq, int k,
 // the first step divides; later steps count (tile, head, sequence) forward.
 // It also tracks the partition units, so that the owner of any tile can be
 // computed.
-template <bool kFB>
+template <bool kFB, int R>
 struct TileWalk {
   int64_t t;                 // current tile number
   int64_t base;              // first tile of the current sequence
@@ -284,7 +297,7 @@ struct TileWalk {
     seq = s;
     len = seq_len(a, r, s);
     lo = len - span_of(len, a.window);
-    nb = tiles_of(len - lo, kTile);
+    nb = tiles_of(len - lo, R);
     if constexpr (kFB) {
       nbp = nb;
       nb += r.nsuf_s != nullptr && s < kLensCache ? r.nsuf_s[s]
@@ -310,8 +323,8 @@ struct TileWalk {
     if constexpr (kFB) {
       locate_tile<kFB>(a, seq, k, len, lo, nbp, tc);
     } else {
-      tc.row0 = lo + k * kTile;
-      tc.rows = min(kTile, len - tc.row0);
+      tc.row0 = lo + k * R;
+      tc.rows = min(R, len - tc.row0);
     }
     tc.seg = int64_t(seq) * a.g + head;
     tc.nb = nb;
@@ -347,13 +360,17 @@ __device__ __forceinline__ void load_q(const DecodeArgs& a, const CUtensorMap* t
   }
 }
 
-// One K or V tile: W/64 boxes of 64 columns x 128 rows, one per half.
-template <int W>
+// One K or V tile: RH x W/64 boxes of 64 columns x 128 rows, one per row
+// half and column half, row half major.
+template <int W, int RH>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int head, int row,
                                           uint64_t pol) {
-  mbar_expect_tx(bar, uint32_t(W / 64) * kHalfBytes);
+  mbar_expect_tx(bar, uint32_t(RH * (W / 64)) * kHalfBytes);
 #pragma unroll
-  for (int hf = 0; hf < W / 64; ++hf) tma_load_3d(dst + hf * kHalfBytes, map, bar, 64 * hf, head, row, pol);
+  for (int rh = 0; rh < RH; ++rh)
+#pragma unroll
+    for (int hf = 0; hf < W / 64; ++hf)
+      tma_load_3d(dst + (rh * (W / 64) + hf) * kHalfBytes, map, bar, 64 * hf, head, row + rh * kTile, pol);
 }
 
 // Fused append: write the step's new row of (sequence, K/V head) into the
@@ -406,10 +423,10 @@ __device__ int pre_issue(const DecodeArgs& a, const Roles& r, const CUtensorMap*
         mv = tm_sv;
       }
     } else {
-      row = seq * a.m_max + len - span_of(len, a.window) + k * kTile;
+      row = seq * a.m_max + len - span_of(len, a.window) + k * C::kRows;
     }
-    load_tile<DK>(r.sbase + C::kK + i * C::kKTileBytes, mk, bar(C::kKFull + i), head, row, pol);
-    load_tile<DV>(r.sbase + C::kV + i * C::kVTileBytes, mv, bar(C::kVFull + i), head, row, pol);
+    load_tile<DK, C::kRowHalves>(r.sbase + C::kK + i * C::kKTileBytes, mk, bar(C::kKFull + i), head, row, pol);
+    load_tile<DV, C::kRowHalves>(r.sbase + C::kV + i * C::kVTileBytes, mv, bar(C::kVFull + i), head, row, pol);
   }
   return npre;
 }
@@ -426,7 +443,7 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
   constexpr uint32_t kRing = kIsK ? C::kK : C::kV;
   auto bar = [&](int id) { return r.sbase + C::kBar + 8u * id; };
   const uint64_t pol = l2_evict_first_policy();
-  TileWalk<kFB> w(a, ws, r);
+  TileWalk<kFB, C::kRows> w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t i = 0;
   int q_issued = -1;
@@ -465,10 +482,10 @@ __device__ void producer(const DecodeArgs& a, const WSched& ws, const Roles& r, 
       row = w.tc.seq * a.m_max + w.tc.row0;
     }
     constexpr int kW = kIsK ? DK : DV;
-    const uint32_t dst = r.sbase + kRing + st * uint32_t(kW / 64) * kHalfBytes;
+    const uint32_t dst = r.sbase + kRing + st * (kIsK ? C::kKTileBytes : C::kVTileBytes);
     if (a.k_new != nullptr && w.tc.k == w.tc.nb - 1)   // this tile holds the sequence's newest row
       append_new_row<kW>(a, kIsK, w.tc.seq, w.tc.head, w.len);
-    load_tile<kW>(dst, map, bar(kFull + st), w.tc.head, row, pol);
+    load_tile<kW, C::kRowHalves>(dst, map, bar(kFull + st), w.tc.head, row, pol);
     if (kIsK) *reinterpret_cast<volatile int*>(r.smem + C::kKIssued) = int(i + 1);
   }
   // Drain: every copy this thread issued has landed before the CTA can exit.
@@ -495,7 +512,7 @@ __device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) 
   const Sched& sc = ws.s;
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   const int n = int(sc.t_end - sc.t_begin);   // tiles of this CTA (fewer than 2^31)
-  TileWalk<kFB> w(a, ws, r);
+  TileWalk<kFB, C::kRows> w(a, ws, r);
   const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);   // K-major, rows of 128 B
   const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
   const uint32_t bar0 = r.sbase + C::kBar;
@@ -512,13 +529,15 @@ __device__ void s_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) 
     // descriptors differ only in their start address (bits 0-13, 16-byte units)
     const uint64_t ka = kdesc0 + uint64_t((uint32_t(kst) * C::kKTileBytes) >> 4);
     const uint64_t qa = qdesc0 + uint64_t((uint32_t(qb) * C::kQBytes) >> 4);
-    const uint32_t d = r.tmem + uint32_t(i & 1) * NP;
+    const uint32_t d = r.tmem + uint32_t(i & 1) * C::kSStride;
 #pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk) {
-      const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-      const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
-      mma_bf16_ss(d, ka + koff, qa + qoff, idesc_qk, kk > 0);
-    }
+    for (int rh = 0; rh < C::kRowHalves; ++rh)
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t koff = ((rh * C::kKHalves + (kk >> 2)) * kHalfBytes + (kk & 3) * 32) >> 4;
+        const uint32_t qoff = ((kk >> 2) * (NP * 128) + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(d + uint32_t(rh) * (kNpv / 2), ka + koff, qa + qoff, idesc_qk, kk > 0);
+      }
     mma_commit(bar(C::kSFull + (i & 1)));
     mma_commit(bar(C::kKEmpty + kst));
     if (w.last) mma_commit(bar(C::kQEmpty + qb));
@@ -540,11 +559,12 @@ __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r)
   const Sched& sc = ws.s;
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int n = int(sc.t_end - sc.t_begin);
-  TileWalk<kFB> w(a, ws, r);
+  TileWalk<kFB, C::kRows> w(a, ws, r);
   // MN-major V^T; its M (V columns) is always 128: with DV = 64 the second
   // 64-column atom points back at the first (leading offset 0), and the
-  // duplicated half of O is never written out.
-  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, DV == 128 ? kHalfBytes : 0u, 1024);
+  // duplicated half of O is never written out; with 256-row tiles it is the
+  // second row half instead.
+  const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, DV == 128 || C::kPair ? kHalfBytes : 0u, 1024);
   const uint64_t pdesc0 = smem_desc_sw128(r.sbase + C::kP, kHalfBytes, 1024);   // MN-major P
   const uint32_t bar0 = r.sbase + C::kBar;
   auto bar = [&](int id) { return bar0 + 8u * uint32_t(id); };
@@ -587,7 +607,8 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
   constexpr uint32_t idesc_qk = idesc_bf16_f32(kTile, NP, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(kTile, kNpv, 1, 1);
   const int n = int(sc.t_end - sc.t_begin);
-  TileWalk<kFB> wq(a, ws, r), wp(a, ws, r);
+  static_assert(!(C::kPair && kFB), "one issuer: 128-row tiles");
+  TileWalk<kFB, C::kRows> wq(a, ws, r), wp(a, ws, r);
   const uint64_t kdesc0 = smem_desc_sw128(r.sbase + C::kK, 16, 1024);
   const uint64_t qdesc0 = smem_desc_sw128(r.sbase + C::kQ, 16, 1024);
   const uint64_t vdesc0 = smem_desc_sw128(r.sbase + C::kV, DV == 128 ? kHalfBytes : 0u, 1024);
@@ -692,15 +713,18 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
   float* lse2 = reinterpret_cast<float*>(r.smem + C::kLse);
   const float c = a.scale * kLog2e;
   const int hq = a.hq;
+  constexpr bool kPair = C::kPair;                 // 256-row tiles: this thread also takes row `row` + 128
+  const uint32_t o_col = kOCol + (kPair && q4 >= 2 ? kNpv / 2 : 0);   // this lane's block of O
   float lpart[CPT];                                // this row's share of the per-head sums
   float sv[CPT];                                   // this row's scaled logits (log2 units)
+  float sv2[CPT];                                  // the same for row `row` + 128 (256-row tiles)
   float mr[CPT];                                   // reference max per head, mirrored from smem
   {   // zero the P buffer: its pad columns must read as zero
     uint4* p = reinterpret_cast<uint4*>(r.smem + C::kP);
     for (int k = tid; k < int(C::kPBytes / 16); k += 256) p[k] = make_uint4(0, 0, 0, 0);
     named_barrier_softmax();
   }
-  TileWalk<kFB> w(a, ws, r);
+  TileWalk<kFB, C::kRows> w(a, ws, r);
   const int64_t n = sc.t_end - sc.t_begin;
   int64_t pv_waited = -1;
   bool failed = false;
@@ -724,7 +748,17 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     const int pb = e.sidx & 1;
     const int64_t slot = partial_slot(blockIdx.x, e.seg);
     float v[CPT];
-    tmem_ld<CPT>(t_lane + kOCol + uint32_t(pb) * kNpv + col0, v);
+    tmem_ld<CPT>(t_lane + o_col + uint32_t(pb) * kNpv + col0, v);
+    if constexpr (kPair) {   // add the second row half's product (lanes 64-127) to the first's
+      float* xb = reinterpret_cast<float*>(r.smem + C::kX);   // [NP][64]
+      if (row >= 64)
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) xb[(col0 + k) * 64 + row - 64] = v[k];
+      named_barrier_softmax();
+      if (row < 64)
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) v[k] += xb[(col0 + k) * 64 + row];
+    }
     if (row >= DV) {
       // columns past DV only repeat the first ones (see the P.V descriptor)
     } else if (e.whole) {
@@ -773,11 +807,20 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     bool ok = wait(C::kSFull + (i & 1), uint32_t(i >> 1) & 1);
     tc_fence_after();
     const bool valid = row < w.tc.rows;
-    tmem_ld<CPT>(t_lane + uint32_t(i & 1) * NP + col0, sv);
+    if constexpr (kPair)
+      tmem_ld_two<CPT>(t_lane + uint32_t(i & 1) * C::kSStride + col0,
+                       t_lane + uint32_t(i & 1) * C::kSStride + kNpv / 2 + col0, sv, sv2);
+    else
+      tmem_ld<CPT>(t_lane + uint32_t(i & 1) * NP + col0, sv);
     tc_fence_before();
     mbar_arrive(bar(C::kSEmpty + (i & 1)));   // S buffer i&1 may take S(i+2)
 #pragma unroll
     for (int k = 0; k < CPT; ++k) sv[k] = valid ? sv[k] * c : -INFINITY;
+    if constexpr (kPair) {
+      const bool valid2 = row + kTile < w.tc.rows;
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) sv2[k] = valid2 ? sv2[k] * c : -INFINITY;
+    }
     if constexpr (kFB) {
       if (w.tc.beam >= 0) {   // a beam's suffix tile counts for that beam's query columns only
         const int cb0 = w.tc.beam * a.q_group_heads, cb1 = cb0 + a.q_group_heads;
@@ -791,7 +834,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
     if (!w.first) {
       float d[CPT];
 #pragma unroll
-      for (int k = 0; k < CPT; ++k) d[k] = (col0 + k < hq) ? sv[k] - mr[k] : -INFINITY;
+      for (int k = 0; k < CPT; ++k) d[k] = (col0 + k < hq) ? (kPair ? fmaxf(sv[k], sv2[k]) : sv[k]) - mr[k] : -INFINITY;
 #pragma unroll
       for (int span = CPT / 2; span >= 1; span >>= 1)
 #pragma unroll
@@ -804,7 +847,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       for (int ch = 0; ch < CPT / W; ++ch) {
         float v[W];
 #pragma unroll
-        for (int k = 0; k < W; ++k) v[k] = sv[ch * W + k];
+        for (int k = 0; k < W; ++k) v[k] = kPair ? fmaxf(sv[ch * W + k], sv2[ch * W + k]) : sv[ch * W + k];
         const float mx = transpose_reduce<W, true>(v, lane);
         if (lane < W) red[gw * NP + col0 + ch * W + lane] = mx;
       }
@@ -837,7 +880,7 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
 #pragma unroll
       for (int k = 0; k < CPT; ++k) lpart[k] *= alpha[col0 + k];
     }
-    uint32_t packed[CPT / 2];
+    uint32_t packed[CPT / 2], packed2[CPT / 2];
 #pragma unroll
     for (int k2 = 0; k2 < CPT / 2; ++k2) {
       const int k = 2 * k2;
@@ -847,6 +890,14 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       lpart[k + 1] += p1;
       __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
       packed[k2] = *reinterpret_cast<uint32_t*>(&b2);
+      if constexpr (kPair) {
+        const float q0 = col0 + k < hq ? ex2_approx(sv2[k] - mr[k]) : 0.f;
+        const float q1 = col0 + k + 1 < hq ? ex2_approx(sv2[k + 1] - mr[k + 1]) : 0.f;
+        lpart[k] += q0;
+        lpart[k + 1] += q1;
+        __nv_bfloat162 c2 = __floats2bfloat162_rn(q0, q1);
+        packed2[k2] = *reinterpret_cast<uint32_t*>(&c2);
+      }
     }
     // O(i-1) must be complete before O is rescaled and before P(i) overwrites
     // the P buffer it read; a ragged tile needs its V rows landed before the
@@ -857,12 +908,12 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       pv_waited = i - 1;
     }
     const int st = int(i % SV);
-    if (w.tc.rows < kTile) ok2 = wait(C::kVFull + st, uint32_t(i / SV) & 1) && ok2;
+    if (w.tc.rows < C::kRows) ok2 = wait(C::kVFull + st, uint32_t(i / SV) & 1) && ok2;
     if (!softmax_barrier_and(ok && ok2)) { failed = true; break; }
     tc_fence_after();
     if (full && !w.first) {
       // rescale the O accumulated so far (thread = output column, its heads)
-      const uint32_t oc = t_lane + kOCol + uint32_t(w.sidx & 1) * kNpv + col0;
+      const uint32_t oc = t_lane + o_col + uint32_t(w.sidx & 1) * kNpv + col0;
       float v[CPT];
       tmem_ld<CPT>(oc, v);
 #pragma unroll
@@ -877,17 +928,29 @@ __device__ void softmax_epilogue(const DecodeArgs& a, const WSched& ws, const Ro
       const int chunk = col0 / 8 + c8;
       *reinterpret_cast<uint4*>(prow + ((chunk ^ (row & 7)) << 4)) =
           make_uint4(packed[c8 * 4], packed[c8 * 4 + 1], packed[c8 * 4 + 2], packed[c8 * 4 + 3]);
+      if constexpr (kPair) {   // row + 128's P in the same line, kNpv/2 columns on
+        const int chunk2 = (kNpv / 2 + col0) / 8 + c8;
+        *reinterpret_cast<uint4*>(prow + ((chunk2 ^ (row & 7)) << 4)) =
+            make_uint4(packed2[c8 * 4], packed2[c8 * 4 + 1], packed2[c8 * 4 + 2], packed2[c8 * 4 + 3]);
+      }
     }
-    if (w.tc.rows < kTile) {
+    if (w.tc.rows < C::kRows) {
       // rows past the sequence end were loaded too; zero them in V so that
       // P = 0 times whatever they hold contributes exactly 0.  Consecutive
       // threads take consecutive 16-byte pieces of a row (no bank conflicts).
+      // A stage is [row half][column half][128 rows][128 bytes].
       unsigned char* vst = r.smem + C::kV + st * C::kVTileBytes;
-      const int nchunks = (kTile - w.tc.rows) * 8 * C::kVHalves;
+      const int nchunks = (C::kRows - w.tc.rows) * 8 * C::kVHalves;
       for (int k = tid; k < nchunks; k += 256) {
         const int vr = w.tc.rows + k / (8 * C::kVHalves), half = (k >> 3) & (C::kVHalves - 1), c16 = k & 7;
-        *reinterpret_cast<uint4*>(vst + half * kHalfBytes + (vr >> 3) * 1024 + (vr & 7) * 128 + c16 * 16) =
-            make_uint4(0, 0, 0, 0);
+        if constexpr (kPair) {
+          const int vh = vr >> 7, vl = vr & 127;
+          *reinterpret_cast<uint4*>(vst + vh * kHalfBytes + (vl >> 3) * 1024 + (vl & 7) * 128 + c16 * 16) =
+              make_uint4(0, 0, 0, 0);
+        } else {
+          *reinterpret_cast<uint4*>(vst + half * kHalfBytes + (vr >> 3) * 1024 + (vr & 7) * 128 + c16 * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
       }
     }
     fence_proxy_async_smem();
@@ -1042,10 +1105,10 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     ws.seq_ubase = 0;
     ws.pre = int(sched_red[0]);
     r.seq0 = seq;   // lens_tab[0] holds this sequence's length
-  } else if (small_schedule_fits(a.b, a.g, a.m_max, kTile, kThreads, kSegUnits,
+  } else if (small_schedule_fits(a.b, a.g, a.m_max, C::kRows, kThreads, kSegUnits,
                                  kFB ? int64_t(a.q_beams) * tiles_of(a.m_s, kTile) : 0)) {
     ws = make_schedule_small<kThreads>(
-        a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
+        a.lens, a.b, a.g, a.m_max, a.window, C::kRows, a.grid, blockIdx.x, a.flags, sched_red, kSegUnits, lens_tab, bs,
         kFB ? reinterpret_cast<int*>(r.smem + C::kNsuf) : nullptr,
         [&](int seq, int head, int k0, int own, int len, int nb) {
           return pre_issue<NP, SK, SV, DK, DV, kFB>(a, r, &tm_k, &tm_v, &tm_q, &tm_sk, &tm_sv, seq, head, k0, own, len, nb);
@@ -1053,7 +1116,7 @@ __device__ __forceinline__ void decode_tc_body(const DecodeArgs& a, const CUtens
     r.seq0 = 0;
     if (kFB) r.nsuf_s = reinterpret_cast<const int*>(r.smem + C::kNsuf);
   } else {
-    ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, a.window, kTile, a.grid, blockIdx.x, a.flags, sched_red,
+    ws = make_schedule_weighted<kThreads>(a.lens, a.b, a.g, a.m_max, a.window, C::kRows, a.grid, blockIdx.x, a.flags, sched_red,
                                           kSegUnits, bs);
     r.seq0 = ws.s.seq;
     if (threadIdx.x < kLensCache && ws.s.seq + int(threadIdx.x) < a.b)   // L1-resident: the schedule just read them
@@ -1186,9 +1249,11 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[one][dev]) {
-    e = kFB  ? cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc))
-        : one ? cudaFuncSetAttribute(decode_tc_one_kernel<NP, SK, SV, DK, DV>,
+    if constexpr (kFB)
+      e = cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(L::kAlloc));
+    else
+      e = one ? cudaFuncSetAttribute(decode_tc_one_kernel<NP, SK, SV, DK, DV>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc))
               : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV, DK, DV>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc));
@@ -1214,7 +1279,7 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq, tsk, tsv);
+  if constexpr (kFB) return cudaLaunchKernelEx(&cfg, decode_tc_beam_kernel<NP, SK, SV, DK, DV>, a, tk, tv, tq, tsk, tsv);
   if (one) {   // one CTA per segment, none idle
     DecodeArgs a1 = a;
     a1.grid = a.b * a.g;
@@ -1243,7 +1308,8 @@ int tc_ctas_per_sm(int) { return 1; }
 int tc_tile_rows() { return kTile; }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
-  if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) || int64_t(a.b) * a.h >= (int64_t(1) << 31))
+  // (row coordinates of a tile's second half reach 256 rows past a tile start)
+  if (int64_t(a.b) * a.m_max >= (int64_t(1) << 31) - 256 || int64_t(a.b) * a.h >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
   if (a.sk != nullptr) {   // beams sharing a prefix, one pass (head size 128)
     if (a.q_beams < 1 || int64_t(a.b) * a.q_beams * a.m_s >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
@@ -1255,7 +1321,12 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   }
   // Ring stages: about 64 KB of K and 96 KB of V tiles whatever the head sizes.
   if (a.dk == 128 && a.d == 128) return launch_hq<2, 3, 128, 128>(a, stream);
-  if (a.dk == 64 && a.d == 64) return launch_hq<4, 6, 64, 64>(a, stream);
+  if (a.dk == 64 && a.d == 64) {   // up to 32 heads per group: 256-row tiles of 32 KB, as at head size 128
+    if (a.hq <= 16) return launch_np<16, 2, 3, 64, 64, false>(a, stream);
+    if (a.hq <= 32) return launch_np<32, 2, 3, 64, 64, false>(a, stream);
+    if (a.hq <= 64) return launch_np<64, 4, 6, 64, 64, false>(a, stream);
+    return cudaErrorInvalidValue;
+  }
   if (a.dk == 128 && a.d == 64) return launch_hq<2, 6, 128, 64>(a, stream);
   if (a.dk == 64 && a.d == 128) return launch_hq<4, 3, 64, 128>(a, stream);
   return cudaErrorInvalidValue;

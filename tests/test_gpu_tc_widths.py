@@ -112,3 +112,41 @@ def test_single_tile_sequences_at_head_size_64():
     ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, wl.g, wl.scale)
     assert np.all(out[2] == 0.0)
     assert_close(out, ref, "bf16", "single tile")
+
+
+PAIR_EDGE_LENS = [1, 127, 128, 129, 255, 256, 257, 383, 384, 385, 511, 512, 513, 767, 768, 769]
+
+
+@pytest.mark.parametrize("hq", [1, 16, 32])
+def test_head_size_64_tiles_of_256_rows(hq):
+    """At head size 64 with up to 32 heads per group a tile is 256 rows (two
+    128-row halves in one pair of products): lengths at and around both
+    half and whole tile edges, segments whole and split between CTAs."""
+    g = 2
+    wl = wl_of(len(PAIR_EDGE_LENS), hq * g, g, 64, 64, 769)
+    lens = np.array(PAIR_EDGE_LENS, np.int32)
+    inp = host_inputs(wl, seed=100 + hq, nan_tail=True, lens=lens)
+    ref, _ = oracle_decode(inp["q_f32"], inp["k_f32"], inp["v_f32"], lens, g, wl.scale)
+    for ctas in (0, 1, 2, 5, 11):
+        out = run(wl, inp, lens, path="tcgen05", num_ctas=ctas)
+        assert_close(out, ref, "bf16", f"h/g={hq} ctas={ctas}")
+
+
+@pytest.mark.parametrize("hq", [8, 32])
+def test_head_size_64_rescales_for_growing_logits(hq):
+    """Logits growing along the sequence move the running maximum within a
+    segment, in either row half of a 256-row tile, so O is rescaled in
+    tensor memory (both halves' blocks of it)."""
+    from grouped_query_attention_mqa_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits
+    wl = wl_of(3, hq, 1, 64, 64, 1100, lo=1100)
+    lens = np.array([1100, 700, 300], np.int32)
+    inp = host_inputs(wl, seed=31, nan_tail=True, lens=lens)
+    ramp = np.linspace(0.0, 6.0, wl.m_max, dtype=np.float32)[None, :, None, None]
+    k = f32_to_bf16_bits(bf16_bits_to_f32(inp["k"]) * 0 + inp["q_f32"][:, :1, None, :] * ramp * 3)
+    kf = bf16_bits_to_f32(k)
+    ref, _ = oracle_decode(inp["q_f32"], kf, inp["v_f32"], lens, 1, wl.scale)
+    for ctas in (0, 1, 4):
+        o = binding.decode(dev(inp["q"], "bf16"), dev(k, "bf16"), dev(inp["v"], "bf16"), torch.from_numpy(lens).cuda(),
+                           wl.scale, path="tcgen05", num_ctas=ctas)
+        torch.cuda.synchronize()
+        assert_close(host64(o), ref, "bf16", f"ramp h/g={hq} ctas={ctas}")
