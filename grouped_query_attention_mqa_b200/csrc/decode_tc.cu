@@ -597,8 +597,8 @@ __device__ void pv_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r)
 // The beam kernel keeps one thread for both streams: S(j) = K Q^T once K(j)
 // (and a segment's Q) has landed and P(j-2) has been consumed (j <= i + 1),
 // O += V^T P(i) once P(i) and V(i) are there; it polls both and issues
-// whichever is ready, with ring stages and phase parities advanced by
-// increments.  (Its walker reads the suffix lengths of every beam; a copy per
+// whichever is ready, P.V first (the softmax waits on it before it can store
+// the next P), with ring stages and phase parities advanced by increments.  (Its walker reads the suffix lengths of every beam; a copy per
 // stream measured slower than one thread serving both.)
 template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r) {
@@ -625,6 +625,28 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
   uint32_t idle_polls = 0;
   while (ip < n) {
     bool progressed = false;
+    if (ip < iq) {
+      const int ob = wp.sidx & 1;
+      if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) && mbar_test(bar(C::kVFull + vst), vph) &&
+          (!wp.first || wp.sidx < 2 || mbar_test(bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))) {
+        tc_fence_after();
+        const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * C::kVTileBytes) >> 4);
+        const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
+        const uint32_t acc0 = wp.first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        mma_commit(bar(C::kOFull));
+        mma_commit(bar(C::kVEmpty + vst));
+        ++ip;
+        if (++vst == SV) {
+          vst = 0;
+          vph ^= 1u;
+        }
+        if (ip < n) wp.next(a, sc);
+        progressed = true;
+      }
+    }
     if (iq < n && iq <= ip + 1) {
       const int qb = wq.sidx & 1;
       if ((!wq.first || mbar_test(bar(C::kQFull + qb), uint32_t(wq.sidx >> 1) & 1)) &&
@@ -648,28 +670,6 @@ __device__ void mma_issuer(const DecodeArgs& a, const WSched& ws, const Roles& r
           kph ^= 1u;
         }
         if (iq < n) wq.next(a, sc);
-        progressed = true;
-      }
-    }
-    if (ip < iq) {
-      const int ob = wp.sidx & 1;
-      if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) && mbar_test(bar(C::kVFull + vst), vph) &&
-          (!wp.first || wp.sidx < 2 || mbar_test(bar(C::kOFree + ob), uint32_t((wp.sidx >> 1) - 1) & 1))) {
-        tc_fence_after();
-        const uint64_t va = vdesc0 + uint64_t((uint32_t(vst) * C::kVTileBytes) >> 4);
-        const uint32_t d = r.tmem + kOCol + uint32_t(ob) * kNpv;
-        const uint32_t acc0 = wp.first ? 0u : 1u;
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16_ss(d, va + ((kk * 2048) >> 4), pdesc0 + ((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-        mma_commit(bar(C::kOFull));
-        mma_commit(bar(C::kVEmpty + vst));
-        ++ip;
-        if (++vst == SV) {
-          vst = 0;
-          vph ^= 1u;
-        }
-        if (ip < n) wp.next(a, sc);
         progressed = true;
       }
     }
