@@ -65,6 +65,9 @@ CASES = [
              scale=1 / math.sqrt(128)),
     Workload("noalloc_gqa", b=3, h=16, g=4, d_k=64, d_v=64, m_max=300, len_lo=40, len_hi=300, dtype="f32",
              scale=1 / math.sqrt(64)),
+    # bf16 at head size 64: the tensor-core kernel's 256-row tiles
+    Workload("noalloc_d64", b=5, h=32, g=2, d_k=64, d_v=64, m_max=900, len_lo=1, len_hi=900, dtype="bf16",
+             scale=1 / math.sqrt(64)),
 ]
 
 
