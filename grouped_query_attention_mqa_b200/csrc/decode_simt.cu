@@ -16,6 +16,7 @@
 // tensor-core kernel, and this one takes fp32, head sizes 32 and 64, and keys
 // and values of different widths (d_k for q and K, d_v for V and o), as the
 // paper's per-head dimensions k and v allow (velog paper review §2.4, §3).
+#include <atomic>
 #include "common.cuh"
 
 namespace mqa {
@@ -333,16 +334,16 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
 // Opt the kernel into large dynamic shared memory once per device.
 template <typename T, int DK, int DV>
 cudaError_t ensure_smem_attr() {
-  static bool done[64] = {false};
+  static std::atomic<bool> done[64];   // per device; any thread may set it (the call is idempotent)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
   int optin = 0;
   e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(decode_simt_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_relaxed);
   return e;
 }
 
@@ -367,11 +368,14 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
 // Resident CTAs per SM for this shared-memory size, cached per (device, h/g).
 template <typename T, int DK, int DV>
 int occupancy_t(int hq) {
-  static int cache[64][129] = {};
+  static std::atomic<int> cache[64][129];   // 0 = not yet known; every thread computes the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   const bool cacheable = dev >= 0 && dev < 64 && hq >= 1 && hq <= 128;
-  if (cacheable && cache[dev][hq] > 0) return cache[dev][hq];
+  if (cacheable) {
+    const int c = cache[dev][hq].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   const size_t smem = SimtLayout<T, DK, DV>::bytes(hq);
   if (ensure_smem_attr<T, DK, DV>() != cudaSuccess) return 1;
   int n = 0;
@@ -379,7 +383,7 @@ int occupancy_t(int hq) {
           cudaSuccess ||
       n < 1)
     n = 1;
-  if (cacheable) cache[dev][hq] = n;
+  if (cacheable) cache[dev][hq].store(n, std::memory_order_relaxed);
   return n;
 }
 

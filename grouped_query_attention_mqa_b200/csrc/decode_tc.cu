@@ -60,6 +60,7 @@
 // Every wait is bounded (one second); on expiry the kernel sets
 // MQA_FLAG_PIPE_TIMEOUT, drains its own copies and MMAs, frees its tensor
 // memory and returns.
+#include <atomic>
 #include <cuda.h>
 
 #include "common.cuh"
@@ -1244,11 +1245,11 @@ template <int NP, int SK, int SV, int DK, int DV, bool kFB>
 cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
   using L = TcCfg<NP, SK, SV, DK, DV>;
   const bool one = !kFB && a.no_merge && int64_t(a.b) * a.g <= a.grid;
-  static bool attr_set[2][64] = {{false}};
+  static std::atomic<bool> attr_set[2][64];   // per kernel and device; setting it twice is harmless
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[one][dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[one][dev].load(std::memory_order_relaxed)) {
     if constexpr (kFB)
       e = cudaFuncSetAttribute(decode_tc_beam_kernel<NP, SK, SV, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(L::kAlloc));
@@ -1258,7 +1259,7 @@ cudaError_t launch_np(const DecodeArgs& a, cudaStream_t stream) {
               : cudaFuncSetAttribute(decode_tc_kernel<NP, SK, SV, DK, DV>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc));
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[one][dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[one][dev].store(true, std::memory_order_relaxed);
   }
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tk, tv, tq, tsk, tsv;

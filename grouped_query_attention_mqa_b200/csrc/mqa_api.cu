@@ -1,5 +1,6 @@
 // The C ABI of libmqa: argument checks, the choice of kernel path and CTA
 // count, and the launches.  No allocation, no synchronisation, no exceptions.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -16,13 +17,16 @@ bool valid_dtype(int dt) { return dt == MQA_F32 || dt == MQA_BF16; }
 
 // SM count of the current device, cached per device.
 int sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];   // 0 = not yet known; every thread computes the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -27,6 +27,7 @@
 //
 // Query tiles are launched longest first (the causal tiles near the end of a
 // sequence carry the most keys), one CTA each.
+#include <atomic>
 #include <cuda.h>
 
 #include "common.cuh"
@@ -412,14 +413,14 @@ cudaError_t launch_prefill_tc(void* o, const void* q, const void* k, const void*
                               cudaStream_t stream) {
   const int hq = h / g;
   if (!prefill_tc_supported(kD, hq) || total >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; setting it twice is harmless
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
     e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kAlloc));
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_relaxed);
   }
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;

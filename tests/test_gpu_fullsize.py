@@ -22,7 +22,8 @@ def _lib():
     binding.load_library()
 
 
-@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k", "mqa_b16_m16k", "mha_b16_m16k"])
+@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k", "mqa_b16_m16k", "mha_b16_m16k",
+                                  "long_mqa_d64_b64_m8k"])
 def test_full_size_step_every_sequence(name):
     wl = WORKLOADS[name]
     inp = device_inputs(wl, seed=3, device="cuda")

@@ -104,7 +104,8 @@ def test_paper_decoder_128_fused_steps(path):
     assert np.array_equal(bits(Kd), K_host) and np.array_equal(bits(Vd), V_host)
 
 
-@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k", "mqa_b16_m16k", "mha_b16_m16k"])
+@pytest.mark.parametrize("name", ["long_mqa_b64_m8k", "gqa8_b32_m32k", "mqa_b16_m16k", "mha_b16_m16k",
+                                  "long_mqa_d64_b64_m8k"])
 def test_full_size_fused_step_every_sequence(name):
     """The bench's step (mqa_decode_append, default path and CTA count) on the
     full-size workloads; every sequence against the oracle, and the caches:
