@@ -10,10 +10,13 @@
 // A CTA takes one 128-row query tile of one (sequence, K/V group): rows are
 // (position, head) pairs, 128 / (h/g) positions times the h/g heads of the
 // group, so every K/V tile it loads feeds all heads of the group (the MQA
-// saving, here in the reuse of each staged tile).  Per 128-key tile:
-//   S = Q K^T      M = 128 rows, N = 128 keys, K = d = 128   (tensor memory)
-//   O += P V       M = 128 rows, N = d = 128, K = 128 keys   (tensor memory)
-// One softmax thread per row holds the tile's 128 logits in registers; its
+// saving, here in the reuse of each staged tile).  Per 64-key tile:
+//   S = Q K^T      M = 128 rows, N = 64 keys, K = d = 128    (tensor memory)
+//   O += P V       M = 128 rows, N = d = 128, K = 64 keys    (tensor memory)
+// Two CTAs share each SM (112 KB of shared memory and 256 tensor-memory
+// columns each): a tile's chain of product, softmax and product costs about
+// the same at 64 keys as at 128, so two independent chains per SM do more.
+// One softmax thread per row holds the tile's 64 logits in registers; its
 // reference max is moved only when a logit exceeds it by more than 8 (log2
 // units), and only then is its row of O rescaled in tensor memory.
 //
@@ -40,18 +43,21 @@ namespace {
 using namespace sm100;
 
 constexpr int kRows = 128;                     // query rows per tile (the MMA M)
-constexpr int kKeys = 128;                     // keys per K/V tile
+constexpr int kKeys = 64;                      // keys per K/V tile
 constexpr int kD = 128;                        // head size
 constexpr int kSK = 2, kSV = 2;                // K and V ring stages
 constexpr int kThreads = 224;                  // 7 warps
+constexpr int kCtasPerSm = 2;                  // two query tiles' pipelines share each SM
 constexpr int kVWarp = 6;
-constexpr uint32_t kHalf = 128 * 128;          // one 64-column half of a 128-row bf16 tile
-constexpr uint32_t kTileBytes = 2 * kHalf;
+constexpr uint32_t kHalf = kRows * 128;        // one 64-column half of the 128-row Q tile
+constexpr uint32_t kHalfKV = kKeys * 128;      // one 64-column half of a K or V tile
+constexpr uint32_t kQBytes = 2 * kHalf, kKVBytes = 2 * kHalfKV;
+constexpr uint32_t kPBytes = kRows * kKeys * 2;   // 128 rows x 64 keys (bf16): one 128-byte swizzle column
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.f;       // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kTmemCols = 512;            // S double buffer at [0, 256), O at [256, 384)
-constexpr uint32_t kOCol = 256;
+constexpr uint32_t kTmemCols = 256;            // S double buffer at [0, 128), O at [128, 256)
+constexpr uint32_t kOCol = 2 * kKeys;
 
 struct Cfg {
   // barriers
@@ -60,16 +66,19 @@ struct Cfg {
                        kDone = kOFull + 1, kNumBars = kDone + 1;
   // shared memory (1024-byte aligned base)
   static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTileBytes;
-  static constexpr uint32_t kV = kK + kSK * kTileBytes;
-  static constexpr uint32_t kP = kV + kSV * kTileBytes;
-  static constexpr uint32_t kBar = kP + kTileBytes;
+  static constexpr uint32_t kK = kQ + kQBytes;
+  static constexpr uint32_t kV = kK + kSK * kKVBytes;
+  static constexpr uint32_t kP = kV + kSV * kKVBytes;
+  static constexpr uint32_t kBar = kP + kPBytes;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kEnd = kAbort + 4;
-  static constexpr uint32_t kAlloc = kEnd + 1024;
+  // No room to align the base at run time: two CTAs per SM leave each at most
+  // (228 KB - 2 x 1 KB reserved) / 2.  The kernel checks that the base it gets
+  // is 1024-byte aligned and refuses to run otherwise.
+  static constexpr uint32_t kAlloc = kEnd;
   static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0, "swizzle atoms need 1024-byte alignment");
-  static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(kAlloc <= (233472 - kCtasPerSm * 1024) / kCtasPerSm, "shared memory budget for two CTAs per SM");
 };
 
 struct PrefillArgs {
@@ -93,7 +102,7 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return p;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using C = Cfg;
@@ -116,9 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-  unsigned char* smem = smem_raw + pad;
-  const uint32_t sbase = raw + pad;
+  if (raw & 1023u) {   // the swizzled tiles need a 1024-byte aligned base (uniform across the CTA)
+    if (a.flags != nullptr && threadIdx.x == 0) atomicOr(a.flags, MQA_FLAG_PIPE_TIMEOUT);
+    return;
+  }
+  unsigned char* smem = smem_raw;
+  const uint32_t sbase = raw;
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kAbort);
   auto bar = [&](int id) { return sbase + C::kBar + 8u * id; };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -159,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool is_k = warp == 0;
       const uint64_t pol = l2_evict_last_policy();   // K/V tiles are read again by the sequence's other tiles
       if (is_k) {
-        mbar_expect_tx(bar(C::kQFull), kTileBytes);
+        mbar_expect_tx(bar(C::kQFull), kQBytes);
         tma_load_3d(sbase + C::kQ, &tm_q, bar(C::kQFull), 0, grp * a.hq, tok0 + p0, l2_evict_first_policy());
         tma_load_3d(sbase + C::kQ + kHalf, &tm_q, bar(C::kQFull), 64, grp * a.hq, tok0 + p0,
                     l2_evict_first_policy());
@@ -176,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (*abort) break;
-        const uint32_t dst = sbase + ring + st * kTileBytes;
-        mbar_expect_tx(bar(full + st), kTileBytes);
+        const uint32_t dst = sbase + ring + st * kKVBytes;
+        mbar_expect_tx(bar(full + st), kKVBytes);
         tma_load_3d(dst, map, bar(full + st), 0, grp, tok0 + k * kKeys, pol);
-        tma_load_3d(dst + kHalf, map, bar(full + st), 64, grp, tok0 + k * kKeys, pol);
+        tma_load_3d(dst + kHalfKV, map, bar(full + st), 64, grp, tok0 + k * kKeys, pol);
       }
       // every copy issued has landed before the CTA may exit
       for (int j = (k - S > 0 ? k - S : 0); j < k; ++j) mbar_wait(bar(full + j % S), uint32_t(j / S) & 1, kTimeoutNs);
@@ -193,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qdesc = smem_desc_sw128(sbase + C::kQ, 16, 1024);        // K-major Q
       const uint64_t kdesc0 = smem_desc_sw128(sbase + C::kK, 16, 1024);       // K-major K (N = keys)
       const uint64_t pdesc = smem_desc_sw128(sbase + C::kP, 16, 1024);        // K-major P (K = keys)
-      const uint64_t vdesc0 = smem_desc_sw128(sbase + C::kV, kHalf, 1024);    // MN-major V (N = d)
+      const uint64_t vdesc0 = smem_desc_sw128(sbase + C::kV, kHalfKV, 1024);  // MN-major V (N = d)
       int iq = 0, ip = 0;
       bool q_ready = false;
       uint32_t idle = 0;
@@ -205,12 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!q_ready) q_ready = mbar_test(bar(C::kQFull), 0);
           if (q_ready && mbar_test(bar(C::kKFull + st), uint32_t(iq / kSK) & 1)) {
             tc_fence_after();
-            const uint64_t ka = kdesc0 + ((st * kTileBytes) >> 4);
+            const uint64_t ka = kdesc0 + ((st * kKVBytes) >> 4);
             const uint32_t d = tmem + uint32_t(iq & 1) * kKeys;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-              mma_bf16_ss(d, qdesc + off, ka + off, idesc_qk, kk > 0);
+              const uint32_t qoff = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+              const uint32_t koff = ((kk >> 2) * kHalfKV + (kk & 3) * 32) >> 4;
+              mma_bf16_ss(d, qdesc + qoff, ka + koff, idesc_qk, kk > 0);
             }
             mma_commit(bar(C::kSFull + (iq & 1)));
             mma_commit(bar(C::kKEmpty + st));
@@ -223,10 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (mbar_test(bar(C::kPFull), uint32_t(ip & 1)) &&
               mbar_test(bar(C::kVFull + st), uint32_t(ip / kSV) & 1)) {
             tc_fence_after();
-            const uint64_t va = vdesc0 + ((st * kTileBytes) >> 4);
+            const uint64_t va = vdesc0 + ((st * kKVBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kKeys / 16; ++kk) {
-              const uint32_t poff = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+              const uint32_t poff = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;   // one 64-key column: kk < 4
               mma_bf16_ss(tmem + kOCol, pdesc + poff, va + ((kk * 2048) >> 4), idesc_pv, (ip > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(bar(C::kOFull));
