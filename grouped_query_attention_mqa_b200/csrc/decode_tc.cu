@@ -1,5 +1,6 @@
 // Split-KV decode attention on the 5th-generation tensor cores (tcgen05),
-// for bf16 caches with head size 128 and up to 64 query heads per K/V head.
+// for bf16 caches with key and value head sizes of 64 or 128 and up to 64
+// query heads per K/V head.
 //
 // Computation ("Fast Transformer Decoding", velog paper review §3; GQA blog
 // "第三站: GQA"): for sequence b and K/V head j the h/g query heads of the

@@ -72,10 +72,11 @@ typedef enum {
 
 /* Kernel path of mqa_decode_ex. */
 typedef enum {
-  MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d = 128, h/g <= 64     */
+  MQA_PATH_AUTO = 0,         /* tensor cores when bf16, d_k and d_v each 64
+                                or 128, h/g <= 64; else CUDA cores           */
   MQA_PATH_SIMT = 1,         /* CUDA-core FFMA path (any dtype, h/g*d <= 4096) */
-  MQA_PATH_TCGEN05 = 2       /* tcgen05 tensor-core path (bf16, d = 128,
-                                h/g <= 64)                                    */
+  MQA_PATH_TCGEN05 = 2       /* tcgen05 tensor-core path (bf16, d_k and d_v
+                                each 64 or 128, h/g <= 64)                    */
 } mqa_path_t;
 
 typedef struct {
@@ -152,8 +153,8 @@ MQA_API size_t mqa_decode_workspace_size(int b, int h, int g, int d_v);
  * Supported: h % g == 0, d_k and d_v in {32, 64, 128}, in any pairing (the
  * paper's per-head key size k and value size v are independent).  The SIMT
  * path takes h/g * d_k <= 4096 and h/g * d_v <= 4096; the tensor-core path
- * bf16 with d_k = d_v = 128 and h/g <= 64 (with d_k != d_v the automatic
- * choice is the SIMT path).  b = 0 is a no-op returning MQA_OK.
+ * bf16 with d_k and d_v each 64 or 128 (any pairing) and h/g <= 64, which the
+ * automatic choice then takes.  b = 0 is a no-op returning MQA_OK.
  * Errors: MQA_ERR_INVALID_ARG (NULL pointer, h % g != 0, non-finite scale,
  * workspace too small or misaligned), MQA_ERR_UNSUPPORTED (head sizes or
  * group widths not built), MQA_ERR_CUDA (launch failure).
